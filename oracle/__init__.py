@@ -1,0 +1,119 @@
+"""fp64 CPU oracle for the DSA sparse-attention step — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The library path never does.
+
+Thin numpy front end over ``dsa_oracle.cpp`` (plain C++, fp64, std::thread
+over query rows).  ``build()`` compiles it with g++; ``lib()`` builds on first
+use when the shared object is missing or stale.
+
+Functions (all inputs are bf16 bit patterns as uint16 arrays):
+  indexer_scores(q_I, w, k_I, kv_start, n_vis, score_ld) -> float64 [T, score_ld]
+  topk(scores, n_vis, topk)                              -> int32 [T, topk]
+  sparse_mla(q, kv, kv_start, idx, scale)                -> (o_lat f64 [T,64,512], lse f64 [T,64])
+  forward(case or arrays, topk, scale)                   -> (o_lat, lse, idx)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa_oracle.cpp")
+_SO = os.path.join(_HERE, "liboracle.so")
+# A test may point the front end at another build of the same source (the
+# mutation test builds deliberately broken copies to show the pins catch them).
+_SO_OVERRIDE = os.environ.get("DSA_ORACLE_SO")
+_lib = None
+
+NTHREADS = os.cpu_count() or 1
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", _SRC, "-o", _SO + ".tmp"]
+        subprocess.check_call(cmd)
+        os.replace(_SO + ".tmp", _SO)
+    return _SO
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if _SO_OVERRIDE:
+            L = ctypes.CDLL(_SO_OVERRIDE)
+        else:
+            build()
+            L = ctypes.CDLL(_SO)
+        P = ctypes.c_void_p
+        L.oracle_indexer_scores.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int64, P, ctypes.c_int]
+        L.oracle_topk.argtypes = [P, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
+        L.oracle_sparse_mla.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P, ctypes.c_int]
+        L.oracle_forward.argtypes = [P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_double, P, P, P, ctypes.c_int]
+        L.oracle_dims.argtypes = [P]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def dims():
+    out = np.zeros(6, np.int32)
+    lib().oracle_dims(_p(out))
+    return tuple(int(x) for x in out)
+
+
+def indexer_scores(q_I, w, k_I, kv_start, n_vis, score_ld=None, nthreads=NTHREADS):
+    q_I, w, k_I = _c(q_I, np.uint16), _c(w, np.uint16), _c(k_I, np.uint16)
+    kv_start, n_vis = _c(kv_start, np.int64), _c(n_vis, np.int32)
+    T = n_vis.shape[0]
+    if score_ld is None:
+        score_ld = int(n_vis.max()) if T else 1
+    out = np.full((T, score_ld), np.nan, np.float64)
+    lib().oracle_indexer_scores(_p(q_I), _p(w), _p(k_I), _p(kv_start), _p(n_vis), T, score_ld, _p(out), nthreads)
+    return out
+
+
+def topk(scores, n_vis, k, nthreads=NTHREADS):
+    scores = _c(scores, np.float64)
+    n_vis = _c(n_vis, np.int32)
+    T = n_vis.shape[0]
+    idx = np.empty((T, k), np.int32)
+    lib().oracle_topk(_p(scores), scores.shape[1], _p(n_vis), T, k, _p(idx), nthreads)
+    return idx
+
+
+def sparse_mla(q, kv, kv_start, idx, scale, nthreads=NTHREADS):
+    q, kv = _c(q, np.uint16), _c(kv, np.uint16)
+    kv_start, idx = _c(kv_start, np.int64), _c(idx, np.int32)
+    T, k = idx.shape
+    o = np.empty((T, 64, 512), np.float64)
+    lse = np.empty((T, 64), np.float64)
+    lib().oracle_sparse_mla(_p(q), _p(kv), _p(kv_start), _p(idx), T, k, float(scale), _p(o), _p(lse), nthreads)
+    return o, lse
+
+
+def forward(q_I, w, k_I, q, kv, kv_start, n_vis, k, scale, nthreads=NTHREADS):
+    q_I, w, k_I = _c(q_I, np.uint16), _c(w, np.uint16), _c(k_I, np.uint16)
+    q, kv = _c(q, np.uint16), _c(kv, np.uint16)
+    kv_start, n_vis = _c(kv_start, np.int64), _c(n_vis, np.int32)
+    T = n_vis.shape[0]
+    o = np.empty((T, 64, 512), np.float64)
+    lse = np.empty((T, 64), np.float64)
+    idx = np.empty((T, k), np.int32)
+    lib().oracle_forward(_p(q_I), _p(w), _p(k_I), _p(q), _p(kv), _p(kv_start), _p(n_vis), T, k,
+                         float(scale), _p(o), _p(lse), _p(idx), nthreads)
+    return o, lse, idx
+
+
+def forward_case(c, scale, nthreads=NTHREADS):
+    return forward(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, c.topk, scale, nthreads)

@@ -1,0 +1,38 @@
+"""Plant plausible mistakes in copies of the oracle source and check that the
+pin suite fails on every one of them (the pins are not vacuous)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "dsa_oracle.cpp")
+
+MUTANTS = {
+    "drop_rope_term": ("sc[j] = (nope + rope) * scale;", "sc[j] = nope * scale;"),
+    "wrong_softmax_scale": ("sc[j] = (nope + rope) * scale;", "sc[j] = (nope + rope) * scale * 0.75;"),
+    "no_normalisation": ("const double p = sc[j] / l;", "const double p = sc[j];"),
+    "lse_sign": ("lse[h] = mx + std::log(l);", "lse[h] = mx - std::log(l);"),
+    "tie_to_higher_position": ("return a < b;", "return a > b;"),
+    "transposed_query_heads": ("dot += q[h * kIdxDim + d] * k[d];", "dot += q[d * kIdxHeads + h] * k[d];"),
+    "single_head_weight": ("wh[h] = widen_bf16(w[h]);", "wh[h] = widen_bf16(w[0]);"),
+    "excludes_self": ("int64_t keep = std::min<int64_t>(topk, n);", "int64_t keep = std::min<int64_t>(topk, n - 1);"),
+    "rope_from_wrong_offset": ("rope += qh[kLatent + d] * r[kLatent + d];", "rope += qh[kLatent + d] * r[d];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    mut = tmp_path / "mut.cpp"
+    mut.write_text(src.replace(old, new))
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["g++", "-O1", "-std=c++17", "-fPIC", "-shared", "-pthread", str(mut), "-o", str(so)])
+    env = dict(os.environ, DSA_ORACLE_SO=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
