@@ -1,0 +1,182 @@
+/*
+ * dsa.h — C ABI of libdsa, the B200 (sm_100a) DSA sparse-attention step:
+ * lightning indexer -> per-row top-k -> sparse MLA attention in latent form.
+ *
+ * What the step computes (pages on the method; page title and section):
+ *  - "GLM 5 DSV3.2 DSA MoE configuration", section 2.2: a lightweight
+ *    indexer scores every query against all of its history and is used only
+ *    to rank; a top-k selector keeps index_topk = 2048 positions; real MLA
+ *    attention runs over those positions only.
+ *  - same page, section 2.1 (config table): index_n_heads 32,
+ *    index_head_dim 128, num_attention_heads 64, kv_lora_rank 512,
+ *    qk_rope_head_dim 64, qk_head_dim 256, index_topk 2048.
+ *  - "DSA + IndexShare explainer", section "DSA full flow": indexer over all
+ *    history -> top-2048 -> softmax over the 2048 and the value mix; the KV
+ *    cache keeps unselected positions for other queries.
+ *  The score and attention formulas (stated on each function) are the
+ *  problem statement's; the pages print none.
+ *
+ * Conventions shared by every entry point
+ *  - Every tensor pointer is a caller-owned DEVICE pointer.  The library never
+ *    allocates or frees device memory; scratch comes from the caller's `ws`.
+ *  - bf16 tensors are passed as their 16-bit patterns (dsa_bf16).
+ *  - Each call enqueues work on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and returns without synchronising.
+ *  - Returns DSA_OK or an error code.  Host-side checks (null pointers,
+ *    alignment, sizes) fail before anything is enqueued.  Per-row problems
+ *    that only the device can see (n_vis or kv_start out of range, an index
+ *    outside the cache) make the kernels skip that row and raise a bit in a
+ *    device status word; a bounded device wait that expires does the same.
+ *    dsa_sync_status() synchronises the stream and reports and clears those
+ *    bits.  dsa_last_error_string() describes the last failure of the
+ *    calling thread.
+ *  - Rows: query row i reads cache rows kv_start[i] .. kv_start[i]+n_vis[i]-1
+ *    of a flat cache of `cache_rows` rows.  The query is at position
+ *    n_vis[i]-1 of its sequence and sees itself (causal: s <= t, n_vis = t+1).
+ *    Positions and indices are relative to kv_start[i].
+ *  - The kernels are built for sm_100a only; other devices get
+ *    DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#define DSA_INDEX_HEADS 32  /* index_n_heads */
+#define DSA_INDEX_DIM 128   /* index_head_dim */
+#define DSA_HEADS 64        /* num_attention_heads */
+#define DSA_LATENT 512      /* kv_lora_rank: width of c_kv and of o_lat */
+#define DSA_ROPE 64         /* qk_rope_head_dim */
+#define DSA_ROW 576         /* DSA_LATENT + DSA_ROPE: one latent-cache row / one latent query */
+#define DSA_MAX_TOPK 2048   /* index_topk */
+
+typedef uint16_t dsa_bf16;             /* bf16 bit pattern */
+typedef struct CUstream_st* dsa_stream_t; /* same type as cudaStream_t */
+
+enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size (host check) */
+  DSA_ERR_WORKSPACE = 2,   /* ws smaller than dsa_workspace_size() */
+  DSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  DSA_ERR_TIMEOUT = 4,     /* a bounded device wait expired (from dsa_sync_status) */
+  DSA_ERR_UNSUPPORTED = 5, /* current device is not sm_100 */
+  DSA_ERR_BAD_ROW = 6      /* a row had n_vis/kv_start/index out of range and was skipped (from dsa_sync_status) */
+};
+
+enum dsa_op {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_MLA = 2,
+  DSA_OP_FORWARD = 3
+};
+
+/*
+ * Bytes of device workspace `op` needs for T query rows, n_vis <= max_n_vis
+ * and the given topk.  Pure host function; 0 means no workspace is needed.
+ */
+DSA_API size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk);
+
+/*
+ * Lightning-indexer scores ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2;
+ * "DSA + IndexShare explainer", section "lightning indexer: low-dimensional
+ * dot products"):
+ *     scores[i, s] = sum_{h<32} w[i,h] * (q_I[i,h,:] . k_I[kv_start[i]+s, :])
+ * for 0 <= s < n_vis[i], computed from bf16 inputs with fp32 accumulation on
+ * the tensor cores.  Columns s >= n_vis[i] of the row are not written.
+ *
+ *  q_I     [T,32,128] bf16, row-major, 16-byte aligned
+ *  w       [T,32]     bf16, 16-byte aligned
+ *  k_I     [cache_rows,128] bf16 (256 B per row), 16-byte aligned
+ *  kv_start[T] int64, n_vis[T] int32 (device); need 1 <= n_vis[i] <= score_ld
+ *          and 0 <= kv_start[i], kv_start[i]+n_vis[i] <= cache_rows
+ *  scores  [T,score_ld] fp32, 16-byte aligned, score_ld % 4 == 0
+ *  ws      >= dsa_workspace_size(DSA_OP_INDEXER, T, score_ld, 0) bytes, 256-byte aligned
+ */
+DSA_API int dsa_indexer_scores(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                       const int64_t* kv_start, const int32_t* n_vis, int T, float* scores, int64_t score_ld,
+                       void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Top-k selector ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2: keep the
+ * index_topk highest-scoring positions; "DSA + IndexShare explainer",
+ * index_topk: 2048).  For row i keeps K = min(topk, n_vis[i]) positions of
+ * scores[i, 0:n_vis[i]] under the total order (score descending, position
+ * ascending: ties go to the lower position; -0.0 equals +0.0), writes them in
+ * ascending position order to idx[i, 0:K] and fills idx[i, K:topk] with -1.
+ * Exact: the kept set is the unique top-K of that order.
+ *
+ *  scores  [T,score_ld] fp32 (16-byte aligned, score_ld % 4 == 0); no NaN
+ *  n_vis   [T] int32 (device), 1 <= n_vis[i] <= score_ld
+ *  idx     [T,topk] int32, 1 <= topk <= 2048
+ */
+DSA_API int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk, int32_t* idx,
+             dsa_stream_t stream);
+
+/*
+ * Sparse MLA attention in latent (absorbed) form over the selected rows
+ * ("DSA + IndexShare explainer", "DSA full flow": full Q.K, softmax and the
+ * value mix over the selected 2048 only; config table: qk_head_dim 256 so the
+ * softmax scale is 1/sqrt(256)).  For row i, head h and the valid entries
+ * s_j = idx[i,j] >= 0:
+ *     S[h,j]   = scale * (q[i,h,0:512] . kv[r_j,0:512] + q[i,h,512:576] . kv[r_j,512:576]),
+ *                r_j = kv_start[i] + s_j
+ *     o_lat[i,h,:] = sum_j softmax_j(S[h,:]) * kv[r_j, 0:512]
+ *     lse[i,h]     = log sum_j exp(S[h,j])           (natural log)
+ * bf16 inputs, fp32 tensor-core accumulation and fp32 softmax.  A row whose
+ * idx holds no valid entry gets o_lat = 0 and lse = -inf.
+ *
+ *  q       [T,64,576] bf16 (q_lat || q_rope), 16-byte aligned
+ *  kv      [cache_rows,576] bf16 (c_kv || k_rope, 1152 B per row), 16-byte aligned
+ *  kv_start[T] int64 (device)
+ *  idx     [T,topk] int32: positions relative to kv_start, -1 = empty slot;
+ *          entries with kv_start+idx >= cache_rows are skipped (status bit)
+ *  o_lat   [T,64,512] fp32, 16-byte aligned; lse [T,64] fp32 or NULL
+ *  ws      >= dsa_workspace_size(DSA_OP_SPARSE_MLA, T, 0, topk) bytes, 256-byte aligned
+ */
+DSA_API int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
+                        const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,
+                        size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * The whole step: indexer -> top-k -> sparse MLA, enqueued on one stream.
+ * Arguments as above; k_I and kv share the row numbering (cache_rows rows).
+ * max_n_vis is a host-side upper bound of n_vis (rows above it are skipped
+ * with a status bit).  idx_out [T,topk] receives the selected positions when
+ * not NULL.  The score matrix is materialised in `ws` when it is small
+ * (T * max_n_vis * 4 bytes within the workspace rule of dsa_workspace_size);
+ * otherwise scores are streamed into the selector and never stored.
+ */
+DSA_API int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q, const dsa_bf16* kv,
+                int64_t cache_rows, const int64_t* kv_start, const int32_t* n_vis, int T, int64_t max_n_vis, int topk,
+                float scale, float* o_lat, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes,
+                dsa_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word of the
+ * current device.  Returns DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_BAD_ROW or
+ * DSA_ERR_CUDA (a sticky CUDA error).
+ */
+DSA_API int dsa_sync_status(dsa_stream_t stream);
+
+/* Message for the calling thread's last failure ("" if none). Never NULL. */
+DSA_API const char* dsa_last_error_string(void);
+
+/* ABI version of this header: 1. */
+DSA_API int dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,331 @@
+// libdsa: the C ABI declared in include/dsa.h, and the only translation unit
+// of the library (the kernels are included below so they share one device
+// status word without relocatable device code).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "dsa.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+#include "indexer.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- per-device state
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  bool prepared = false;
+  int sm_count = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+    d.probed = true;
+  }
+  if (!d.supported) return fail(DSA_ERR_UNSUPPORTED, "libdsa is built for sm_100a; device %d is not", dev);
+  if (!d.prepared) {
+    if ((e = dsa::prepare_indexer()) != cudaSuccess) return cuda_fail(e, "indexer smem opt-in");
+    if ((e = dsa::prepare_sparse_mla()) != cudaSuccess) return cuda_fail(e, "sparse MLA smem opt-in");
+    d.prepared = true;
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+unsigned long long wait_limit_ns() {
+  static unsigned long long v = [] {
+    const char* s = std::getenv("DSA_WAIT_LIMIT_NS");
+    if (s && *s) {
+      unsigned long long x = std::strtoull(s, nullptr, 10);
+      if (x > 0) return x;
+    }
+    return 1500000000ull;  // 1.5 s per wait
+  }();
+  return v;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return EncodeTiledFn(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] tensor map with a box of [box_rows, 64] and 128-byte swizzle.
+int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- sizes
+int64_t score_ld_for(int64_t max_n_vis) { return (max_n_vis + 3) / 4 * 4; }
+
+size_t ws_indexer(int T) { return align_up(dsa::indexer_plan_bytes(T), 256); }
+
+size_t ws_forward(int T, int64_t max_n_vis, int topk) {
+  return ws_indexer(T) + align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256) +
+         align_up(size_t(T) * size_t(topk) * 4, 256);
+}
+
+int pick_qmax(int T) {
+  const char* s = std::getenv("DSA_INDEXER_QMAX");
+  if (s && *s) {
+    int v = std::atoi(s);
+    if (v == 1 || v == 4 || v == 8) return v;
+  }
+  return T >= 5 ? 8 : (T >= 2 ? 4 : 1);
+}
+
+int check_common_rows(int T, int64_t cache_rows, const void* kv_start) {
+  if (T < 0) return fail(DSA_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+  if (cache_rows < 1 || cache_rows > INT32_MAX)
+    return fail(DSA_ERR_INVALID_ARG, "cache_rows must lie in [1, 2^31-1] (got %lld)", (long long)cache_rows);
+  if (T > 0 && !kv_start) return fail(DSA_ERR_INVALID_ARG, "kv_start is NULL");
+  if (!aligned(kv_start, 8)) return fail(DSA_ERR_INVALID_ARG, "kv_start must be 8-byte aligned");
+  return DSA_OK;
+}
+
+int run_indexer(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                const int64_t* kv_start, const int32_t* n_vis, int T, float* scores, int64_t score_ld, void* plan,
+                dsa_stream_t stream, int sm_count) {
+  int qmax = pick_qmax(T);
+  CUtensorMap tk, tq;
+  int rc = make_tmap_bf16(&tk, k_I, DSA_INDEX_DIM, uint64_t(cache_rows), 128);
+  if (rc) return rc;
+  rc = make_tmap_bf16(&tq, q_I, DSA_INDEX_DIM, uint64_t(T) * DSA_INDEX_HEADS, 32);
+  if (rc) return rc;
+  dsa::IndexerLaunch p{};
+  p.q_I = q_I;
+  p.w = w;
+  p.k_I = k_I;
+  p.cache_rows = cache_rows;
+  p.kv_start = kv_start;
+  p.n_vis = n_vis;
+  p.T = T;
+  p.scores = scores;
+  p.score_ld = score_ld;
+  p.plan = plan;
+  p.qmax = qmax;
+  // Wave sweep when many query tiles share a key set larger than a good part of L2:
+  // all CTAs then walk the keys in step and each key tile leaves HBM about once per wave.
+  const int n_tiles_min = (T + qmax - 1) / qmax;
+  p.sweep = (n_tiles_min >= sm_count && score_ld * 256 > (64ll << 20)) ? dsa::kSweepWave : dsa::kSweepSplit;
+  if (const char* sw = std::getenv("DSA_INDEXER_SWEEP")) {
+    if (!std::strcmp(sw, "wave")) p.sweep = dsa::kSweepWave;
+    if (!std::strcmp(sw, "split")) p.sweep = dsa::kSweepSplit;
+  }
+  p.grid = sm_count;
+  p.wait_ns = wait_limit_ns();
+  p.stream = stream;
+  cudaError_t e = dsa::launch_indexer(p, tk, tq);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_abi_version(void) { return 1; }
+
+const char* dsa_last_error_string(void) { return t_err.c_str(); }
+
+size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
+  if (T < 0) T = 0;
+  if (max_n_vis < 0) max_n_vis = 0;
+  if (topk < 0) topk = 0;
+  switch (op) {
+    case DSA_OP_INDEXER: return ws_indexer(T);
+    case DSA_OP_TOPK: return 0;
+    case DSA_OP_SPARSE_MLA: return 0;
+    case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
+    default: return 0;
+  }
+}
+
+int dsa_indexer_scores(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                       const int64_t* kv_start, const int32_t* n_vis, int T, float* scores, int64_t score_ld,
+                       void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (T == 0) return DSA_OK;
+  if (!q_I || !w || !k_I || !n_vis || !scores || !ws)
+    return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_I, 16) || !aligned(w, 16) || !aligned(k_I, 16) || !aligned(scores, 16) || !aligned(n_vis, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q_I, w, k_I, scores must be 16-byte aligned and n_vis 4-byte aligned");
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (score_ld < 4 || score_ld % 4 != 0) return fail(DSA_ERR_INVALID_ARG, "score_ld must be a positive multiple of 4");
+  if (int64_t(T) * DSA_INDEX_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
+  if (ws_bytes < ws_indexer(T))
+    return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, ws_indexer(T));
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, score_ld, ws, stream, dev->sm_count);
+}
+
+int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk, int32_t* idx,
+             dsa_stream_t stream) {
+  t_err.clear();
+  if (T < 0) return fail(DSA_ERR_INVALID_ARG, "T must be >= 0");
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
+  if (T == 0) return DSA_OK;
+  if (!scores || !n_vis || !idx) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(scores, 16) || !aligned(n_vis, 4) || !aligned(idx, 4))
+    return fail(DSA_ERR_INVALID_ARG, "scores must be 16-byte aligned, n_vis and idx 4-byte aligned");
+  if (score_ld < 4 || score_ld % 4 != 0) return fail(DSA_ERR_INVALID_ARG, "score_ld must be a positive multiple of 4");
+  if (score_ld > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "score_ld too large");
+  DeviceState* dev = nullptr;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  cudaError_t e = dsa::launch_topk(scores, score_ld, n_vis, T, topk, idx, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  return DSA_OK;
+}
+
+int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
+                        const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,
+                        size_t ws_bytes, dsa_stream_t stream) {
+  t_err.clear();
+  (void)ws;
+  (void)ws_bytes;
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
+  if (T == 0) return DSA_OK;
+  if (!q || !kv || !idx || !o_lat) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o_lat, 16) || !aligned(idx, 4) || !aligned(lse, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q, kv, o_lat must be 16-byte aligned; idx, lse 4-byte aligned");
+  if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  dsa::MlaLaunch p{q, kv, cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, wait_limit_ns(), stream};
+  cudaError_t e = dsa::launch_sparse_mla(p);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
+  return DSA_OK;
+}
+
+int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q, const dsa_bf16* kv,
+                int64_t cache_rows, const int64_t* kv_start, const int32_t* n_vis, int T, int64_t max_n_vis, int topk,
+                float scale, float* o_lat, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes,
+                dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
+  if (T == 0) return DSA_OK;
+  if (max_n_vis < 1 || max_n_vis > cache_rows)
+    return fail(DSA_ERR_INVALID_ARG, "max_n_vis must lie in [1, cache_rows]");
+  if (!q_I || !w || !k_I || !q || !kv || !n_vis || !o_lat || !ws)
+    return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_I, 16) || !aligned(w, 16) || !aligned(k_I, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
+      !aligned(o_lat, 16) || !aligned(n_vis, 4) || !aligned(lse, 4) || !aligned(idx_out, 4))
+    return fail(DSA_ERR_INVALID_ARG, "tensor pointers misaligned (bf16/o_lat 16 B, n_vis/lse/idx 4 B)");
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  const size_t need = ws_forward(T, max_n_vis, topk);
+  if (ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, need);
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+
+  const int64_t ld = score_ld_for(max_n_vis);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* plan = base;
+  float* scores = reinterpret_cast<float*>(base + ws_indexer(T));
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(base + ws_indexer(T) + align_up(size_t(T) * size_t(ld) * 4, 256));
+  int32_t* idx = idx_out ? idx_out : idx_ws;
+
+  if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, ld, plan, stream, dev->sm_count)))
+    return rc;
+  cudaError_t e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  dsa::MlaLaunch p{q, kv, cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, wait_limit_ns(), stream};
+  e = dsa::launch_sparse_mla(p);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
+  return DSA_OK;
+}
+
+int dsa_sync_status(dsa_stream_t stream) {
+  t_err.clear();
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int st = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&st, dsa::g_status, sizeof st);
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (st) {
+    e = cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  }
+  if (st & dsa::kStatusTimeout) return fail(DSA_ERR_TIMEOUT, "a bounded device wait expired (status 0x%x)", st);
+  if (st & (dsa::kStatusBadRow | dsa::kStatusOverflow))
+    return fail(DSA_ERR_BAD_ROW, "a row was skipped: n_vis, kv_start or an index out of range (status 0x%x)", st);
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,442 @@
+// Lightning-indexer scores on the 5th-generation tensor cores.
+//
+//   scores[i, s] = sum_{h<32} w[i,h] * (q_I[i,h,:] . k_I[kv_start[i]+s, :])
+//
+// ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2: a light scorer of every
+// query against all history, 32 heads x 128 dims; the per-head weighting and
+// head sum are the problem statement's.)
+//
+// Swap-AB formulation: one tcgen05.mma of M = 128 keys (TMEM lanes) x
+// N = 32 * nq (heads x queries of one query tile) x K = 128 produces every
+// head's dot product for 128 keys and up to 8 queries that share the
+// sequence.  Keys arrive by TMA (two 64-column boxes, 128-byte swizzle) into
+// a STAGES-deep ring; the query tile's q_I sits in its own buffer.  In the
+// epilogue each of 128 threads owns one key row: it reads that row's 32 head
+// columns per query from TMEM and reduces them with w into one fp32 score,
+// so the head reduction needs no cross-thread traffic.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
+// and MMA issuer, warps 2..5 = epilogue.  Persistent grid.
+#pragma once
+#include <cuda.h>
+
+#include "block_scan.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kKeysPerUnit = 128;
+constexpr int kStageBytes = kKeysPerUnit * 128 * 2;  // 32 KB: 128 keys x 128 dims bf16
+constexpr int kHalfKeyBytes = kStageBytes / 2;       // one 64-column box
+constexpr int kQRowsPerQuery = 32;                   // heads
+constexpr int kQBoxBytes = kQRowsPerQuery * 64 * 2;  // 4 KB: one query, one 64-column half
+
+// ------------------------------------------------------------------ plan kernel
+__global__ void __launch_bounds__(1024) indexer_plan_kernel(const int64_t* __restrict__ kv_start,
+                                                            const int32_t* __restrict__ n_vis, int T, int qmax,
+                                                            int64_t score_ld, int64_t cache_rows,
+                                                            PlanHeader* __restrict__ hdr,
+                                                            PlanTile* __restrict__ tiles) {
+  __shared__ int sc_i[33];
+  __shared__ long long sc_l[33];
+  __shared__ int carry_seg_s;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < T; i += blockDim.x) {
+    PlanTile z;
+    z.q0 = 0;
+    z.nq = 0;
+    z.units = 0;
+    z.pad = 0;
+    z.kv_start = 0;
+    z.unit_begin = 0;
+    tiles[i] = z;
+  }
+  __syncthreads();
+
+  auto row_ok = [&](int i, long long& ks, int& nv) {
+    ks = kv_start[i];
+    nv = n_vis[i];
+    return nv >= 1 && nv <= score_ld && ks >= 0 && ks + nv <= cache_rows;
+  };
+
+  int carry_seg = -1, carry_tiles = 0;
+  for (int base = 0; base < T; base += blockDim.x) {
+    const int i = base + tid;
+    const bool in = i < T;
+    long long ks = 0;
+    int nv = 0;
+    bool ok = false, head = false;
+    if (in) {
+      ok = row_ok(i, ks, nv);
+      if (!ok) raise_status(kStatusBadRow);
+      if (i == 0) {
+        head = true;
+      } else {
+        long long ksp;
+        int nvp;
+        bool okp = row_ok(i - 1, ksp, nvp);
+        head = !ok || !okp || ks != ksp;
+      }
+    }
+    int seg = block_inclusive_max<int>(head ? i : -1, sc_i, -1);
+    seg = seg > carry_seg ? seg : carry_seg;
+    bool tstart = false;
+    int q0 = 0;
+    if (in) {
+      q0 = seg + ((i - seg) / qmax) * qmax;
+      tstart = (q0 == i);
+    }
+    int total = 0;
+    int excl = block_exclusive_sum<int>(tstart ? 1 : 0, sc_i, &total);
+    if (in) {
+      const int tile = carry_tiles + excl - (tstart ? 0 : 1);
+      if (tstart) {
+        tiles[tile].q0 = i;
+        tiles[tile].kv_start = ks;
+      }
+      atomicMax(&tiles[tile].nq, i - q0 + 1);
+      atomicMax(&tiles[tile].units, ok ? (nv + kKeysPerUnit - 1) / kKeysPerUnit : 0);
+    }
+    const int last = (T - 1 - base) < int(blockDim.x - 1) ? (T - 1 - base) : int(blockDim.x - 1);
+    if (tid == last) carry_seg_s = seg;
+    __syncthreads();
+    carry_seg = carry_seg_s;
+    carry_tiles += total;
+    __syncthreads();
+  }
+  __threadfence_block();
+  __syncthreads();
+
+  const int n_tiles = carry_tiles;
+  long long carry = 0;
+  for (int base = 0; base < n_tiles; base += blockDim.x) {
+    const int j = base + tid;
+    long long u = j < n_tiles ? (long long)tiles[j].units : 0;
+    long long total = 0;
+    long long ex = block_exclusive_sum<long long>(u, sc_l, &total);
+    if (j < n_tiles) tiles[j].unit_begin = carry + ex;
+    carry += total;
+  }
+  if (tid == 0) {
+    hdr->total_units = carry;
+    hdr->n_tiles = n_tiles;
+  }
+}
+
+// ------------------------------------------------------------------ unit iterator
+// Every role of the main kernel walks the same sequence of (query tile, key tile).
+struct UnitIter {
+  const PlanTile* tiles;
+  int n_tiles;
+  int sweep;
+  int tile;
+  int kt;
+  long long left;  // units left (split sweep)
+  PlanTile cur;
+
+  __device__ bool load_tile(int j) {
+    while (j < n_tiles && tiles[j].units == 0) j += (sweep == kSweepWave ? int(gridDim.x) : 1);
+    if (j >= n_tiles) return false;
+    tile = j;
+    cur = tiles[j];
+    return true;
+  }
+  __device__ bool begin(const PlanHeader* hdr, const PlanTile* t) {
+    tiles = t;
+    n_tiles = hdr->n_tiles;
+    const long long U = hdr->total_units;
+    kt = 0;
+    if (sweep == kSweepWave) {
+      left = 1;
+      return load_tile(int(blockIdx.x));
+    }
+    const long long G = gridDim.x;
+    const long long b = U * (long long)blockIdx.x / G, e = U * (long long)(blockIdx.x + 1) / G;
+    left = e - b;
+    if (left <= 0) return false;
+    // last tile whose unit_begin <= b
+    int lo = 0, hi = n_tiles - 1;
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (tiles[mid].unit_begin <= b) lo = mid;
+      else hi = mid - 1;
+    }
+    if (!load_tile(lo)) return false;
+    kt = int(b - cur.unit_begin);
+    return true;
+  }
+  __device__ bool next() {
+    ++kt;
+    if (sweep != kSweepWave) {
+      if (--left <= 0) return false;
+    }
+    if (kt < cur.units) return true;
+    kt = 0;
+    return load_tile(tile + (sweep == kSweepWave ? int(gridDim.x) : 1));
+  }
+};
+
+// ------------------------------------------------------------------ main kernel
+template <int QMAX, int STAGES, int QBUF>
+struct IdxSmem {
+  static constexpr int kQBufBytes = QMAX * 2 * kQBoxBytes;  // two halves
+  static constexpr int kKeysOff = 0;
+  static constexpr int kQOff = STAGES * kStageBytes;
+  static constexpr int kWOff = kQOff + QBUF * kQBufBytes;             // float w[QMAX*32]
+  static constexpr int kNvOff = kWOff + QMAX * 32 * 4;                // int n_vis[QMAX]
+  static constexpr int kBarOff = (kNvOff + QMAX * 4 + 7) & ~7;
+  static constexpr int kNumBars = 2 * STAGES + 2 * QBUF + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;             // tmem slot, abort flag
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;                        // slack for 1 KB alignment
+  static constexpr int kAccCols = 32 * QMAX;
+  static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : (2 * kAccCols);
+};
+
+template <int QMAX, int STAGES, int QBUF>
+__global__ void __launch_bounds__(192, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                   const uint16_t* __restrict__ w, const int32_t* __restrict__ n_vis,
+                   const PlanHeader* __restrict__ hdr, const PlanTile* __restrict__ tiles, float* __restrict__ scores,
+                   int64_t score_ld, int sweep, WaitLimit lim) {
+  using L = IdxSmem<QMAX, STAGES, QBUF>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* w_s = reinterpret_cast<float*>(smem + L::kWOff);
+  int* nv_s = reinterpret_cast<int*>(smem + L::kNvOff);
+  const uint32_t bar0 = sbase + L::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto qfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto qempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + QBUF + b); };
+  auto afull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * QBUF + b); };
+  auto aempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 * QBUF + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * QBUF + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < QBUF; ++b) {
+      mbar_init(qfull_bar(b), 1);
+      mbar_init(qempty_bar(b), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(afull_bar(b), 1);
+      mbar_init(aempty_bar(b), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      UnitIter it;
+      it.sweep = sweep;
+      int stage = 0, qb = -1, prev_tile = -1;
+      uint32_t phase = 0;
+      uint32_t qphase[QBUF];
+      for (int b = 0; b < QBUF; ++b) qphase[b] = 0;
+      int issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      bool ok = it.begin(hdr, tiles);
+      while (ok) {
+        if (it.tile != prev_tile) {
+          qb = (qb + 1) % QBUF;
+          if (!mbar_wait(qempty_bar(qb), qphase[qb] ^ 1u, lim, abort_flag)) break;
+          const int nq = it.cur.nq;
+          mbar_arrive_expect_tx(qfull_bar(qb), uint32_t(nq) * 2u * kQBoxBytes);
+          const uint32_t qdst = sbase + L::kQOff + qb * L::kQBufBytes;
+          for (int qi = 0; qi < nq; ++qi) {
+            const int y = (it.cur.q0 + qi) * kQRowsPerQuery;
+            tma_load_2d(qdst + qi * kQBoxBytes, &tmap_q, qfull_bar(qb), 0, y);
+            tma_load_2d(qdst + QMAX * kQBoxBytes + qi * kQBoxBytes, &tmap_q, qfull_bar(qb), 64, y);
+          }
+          qphase[qb] ^= 1u;
+          prev_tile = it.tile;
+        }
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, lim, abort_flag)) break;
+        mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
+        const int y = int(it.cur.kv_start + (long long)it.kt * kKeysPerUnit);
+        const uint32_t kdst = sbase + L::kKeysOff + stage * kStageBytes;
+        tma_load_2d(kdst, &tmap_k, full_bar(stage), 0, y);
+        tma_load_2d(kdst + kHalfKeyBytes, &tmap_k, full_bar(stage), 64, y);
+        ++issued[stage];
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        ok = it.next();
+      }
+      // Drain: every key stage we loaded must have landed before the CTA exits.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > 0) mbar_wait(full_bar(s), uint32_t((issued[s] - 1) & 1), lim, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      UnitIter it;
+      it.sweep = sweep;
+      int stage = 0, qb = -1, prev_tile = -1, ab = 0;
+      uint32_t phase = 0, aphase = 0;
+      uint32_t qphase[QBUF];
+      for (int b = 0; b < QBUF; ++b) qphase[b] = 0;
+      bool ok = it.begin(hdr, tiles);
+      while (ok) {
+        if (it.tile != prev_tile) {
+          if (qb >= 0) mma_commit(qempty_bar(qb));  // previous query buffer free once its MMAs finish
+          qb = (qb + 1) % QBUF;
+          if (!mbar_wait(qfull_bar(qb), qphase[qb], lim, abort_flag)) break;
+          qphase[qb] ^= 1u;
+          prev_tile = it.tile;
+        }
+        if (!mbar_wait(aempty_bar(ab), aphase ^ 1u, lim, abort_flag)) break;
+        if (!mbar_wait(full_bar(stage), phase, lim, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16(128, 32 * it.cur.nq, 0, 0);
+        const uint32_t kaddr = sbase + L::kKeysOff + stage * kStageBytes;
+        const uint32_t qaddr = sbase + L::kQOff + qb * L::kQBufBytes;
+        const uint32_t d_tmem = tmem_base + uint32_t(ab * L::kAccCols);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t koff = uint32_t((k >> 2) * kHalfKeyBytes + (k & 3) * 32);
+          const uint32_t qoff = uint32_t((k >> 2) * QMAX * kQBoxBytes + (k & 3) * 32);
+          const uint64_t ad = smem_desc(kaddr + koff, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(qaddr + qoff, 16, 1024, kSwizzle128B);
+          mma_bf16_ss(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        mma_commit(empty_bar(stage));
+        mma_commit(afull_bar(ab));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        if (++ab == 2) {
+          ab = 0;
+          aphase ^= 1u;
+        }
+        ok = it.next();
+      }
+      // Drain: wait until every MMA issued above has completed.
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, lim, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127
+    UnitIter it;
+    it.sweep = sweep;
+    int prev_tile = -1, ab = 0;
+    uint32_t aphase = 0;
+    bool ok = it.begin(hdr, tiles);
+    while (ok) {
+      const int nq = it.cur.nq;
+      if (it.tile != prev_tile) {
+        named_bar_sync(1, 128);
+        for (int e = et; e < nq * 32; e += 128)
+          w_s[e] = bf16_bits_to_float(w[(long long)it.cur.q0 * 32 + e]);
+        if (et < nq) nv_s[et] = n_vis[it.cur.q0 + et];
+        named_bar_sync(1, 128);
+        prev_tile = it.tile;
+      }
+      if (!mbar_wait(afull_bar(ab), aphase, lim, abort_flag)) break;
+      tc_fence_after();
+      const long long s = (long long)it.kt * kKeysPerUnit + row;
+      const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
+      for (int qi = 0; qi < nq; ++qi) {
+        float v[32];
+        tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
+        const float* wq = w_s + qi * 32;
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) acc = fmaf(wq[h], v[h], acc);
+        if (s < nv_s[qi]) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = acc;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(aempty_bar(ab));
+      if (++ab == 2) {
+        ab = 0;
+        aphase ^= 1u;
+      }
+      ok = it.next();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+template <int QMAX, int STAGES, int QBUF>
+cudaError_t set_smem_attr() {
+  using L = IdxSmem<QMAX, STAGES, QBUF>;
+  static_assert(L::kAlloc <= 232448, "indexer shared memory exceeds the per-CTA limit");
+  return cudaFuncSetAttribute(indexer_kernel<QMAX, STAGES, QBUF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              L::kAlloc);
+}
+
+template <int QMAX, int STAGES, int QBUF>
+cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUtensorMap& tq) {
+  using L = IdxSmem<QMAX, STAGES, QBUF>;
+  auto* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
+  auto* tiles = reinterpret_cast<const PlanTile*>(reinterpret_cast<const uint8_t*>(p.plan) + sizeof(PlanHeader));
+  indexer_kernel<QMAX, STAGES, QBUF><<<p.grid, 192, L::kAlloc, p.stream>>>(
+      tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, WaitLimit{p.wait_ns});
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t prepare_indexer() {
+  cudaError_t e;
+  if ((e = set_smem_attr<1, 6, 2>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<4, 4, 2>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<8, 4, 1>()) != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+cudaError_t launch_indexer(const IndexerLaunch& p, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q) {
+  if (p.T <= 0) return cudaSuccess;
+  auto* hdr = reinterpret_cast<PlanHeader*>(p.plan);
+  auto* tiles = reinterpret_cast<PlanTile*>(reinterpret_cast<uint8_t*>(p.plan) + sizeof(PlanHeader));
+  indexer_plan_kernel<<<1, 1024, 0, p.stream>>>(p.kv_start, p.n_vis, p.T, p.qmax, p.score_ld, p.cache_rows, hdr,
+                                                tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  switch (p.qmax) {
+    case 1: return launch_main<1, 6, 2>(p, tmap_k, tmap_q);
+    case 4: return launch_main<4, 4, 2>(p, tmap_k, tmap_q);
+    case 8: return launch_main<8, 4, 1>(p, tmap_k, tmap_q);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dsa

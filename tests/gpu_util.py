@@ -1,0 +1,112 @@
+"""Helpers shared by the GPU tests: move seeded cases to the device and
+compare the CUDA path with the oracle under the stated tolerances."""
+import numpy as np
+
+from indexer_selected_sparse_dsa_b200 import binding as B
+from indexer_selected_sparse_dsa_b200 import workloads as wl
+
+SCALE = wl.SCALE
+IDX_TOL_REL = 2e-2        # indexer: |dI| <= 2e-2 * max|I|
+SET_TOL_REL = 1e-3        # selection may differ only within 1e-3 * max|I| of the k-th score
+ATT_MAX_ABS = 2e-2        # attention: max-abs
+ATT_REL_L2 = 5e-3         # attention: relative L2
+
+
+def to_dev(c):
+    import torch
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    return dict(q_I=bf(c.q_I), w=bf(c.w), k_I=bf(c.k_I), q=bf(c.q), kv=bf(c.kv),
+                kv_start=torch.from_numpy(np.asarray(c.kv_start, np.int64)).cuda(),
+                n_vis=torch.from_numpy(np.asarray(c.n_vis, np.int32)).cuda())
+
+
+def gpu_scores(d, score_ld, fill=float("nan")):
+    import torch
+    T = d["n_vis"].shape[0]
+    scores = torch.full((T, score_ld), fill, dtype=torch.float32, device="cuda")
+    ws = B.workspace(B.DSA_OP_INDEXER, T, score_ld, 0)
+    B.dsa_indexer_scores(d["q_I"], d["w"], d["k_I"], d["kv_start"], d["n_vis"], scores, ws)
+    B.dsa_sync_status()
+    return scores
+
+
+def gpu_topk(scores_np_f32, n_vis, k):
+    import torch
+    s = torch.from_numpy(np.ascontiguousarray(scores_np_f32, np.float32)).cuda()
+    nv = torch.from_numpy(np.asarray(n_vis, np.int32)).cuda()
+    idx = torch.empty((s.shape[0], k), dtype=torch.int32, device="cuda")
+    B.dsa_topk(s, nv, k, idx)
+    B.dsa_sync_status()
+    return idx.cpu().numpy()
+
+
+def gpu_attention(d, idx_np, scale=SCALE):
+    import torch
+    T, k = idx_np.shape
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, np.int32)).cuda()
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    B.dsa_sparse_mla_attn(d["q"], d["kv"], d["kv_start"], idx, scale, o, lse)
+    B.dsa_sync_status()
+    return o.cpu().numpy(), lse.cpu().numpy()
+
+
+def gpu_forward(d, max_n_vis, k, scale=SCALE):
+    import torch
+    T = d["n_vis"].shape[0]
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    ws = B.workspace(B.DSA_OP_FORWARD, T, max_n_vis, k)
+    B.dsa_forward(d["q_I"], d["w"], d["k_I"], d["q"], d["kv"], d["kv_start"], d["n_vis"], max_n_vis, k, scale,
+                  o, lse, idx, ws)
+    B.dsa_sync_status()
+    return o.cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+
+
+def assert_scores_close(got, ref, n_vis):
+    for i, n in enumerate(n_vis):
+        r = ref[i, :n]
+        g = got[i, :n].astype(np.float64)
+        tol = IDX_TOL_REL * np.max(np.abs(r))
+        err = np.max(np.abs(g - r))
+        assert np.isfinite(g).all(), f"row {i}: non-finite score"
+        assert err <= tol, f"row {i}: max |dI| {err:.3e} > {tol:.3e}"
+
+
+def assert_attention_close(o, lse, o_ref, lse_ref, rows=None):
+    rows = range(o.shape[0]) if rows is None else rows
+    for i in rows:
+        d = o[i].astype(np.float64) - o_ref[i]
+        mabs = np.max(np.abs(d))
+        rel = np.linalg.norm(d) / max(np.linalg.norm(o_ref[i]), 1e-30)
+        assert mabs <= ATT_MAX_ABS, f"row {i}: max-abs {mabs:.3e}"
+        assert rel <= ATT_REL_L2, f"row {i}: rel-L2 {rel:.3e}"
+        fin = np.isfinite(lse_ref[i])
+        assert np.array_equal(fin, np.isfinite(lse[i])), f"row {i}: lse finiteness differs"
+        if fin.any():
+            assert np.max(np.abs(lse[i][fin] - lse_ref[i][fin])) <= ATT_MAX_ABS, f"row {i}: lse"
+
+
+def assert_selection_ok(idx_gpu, scores_ref, n_vis, k):
+    """The GPU's kept set may differ from the oracle's only at positions whose
+    oracle score lies within 1e-3 * max|I| of the oracle's k-th score; and it
+    must be a valid selection: ascending, -1 padded, size min(k, n_vis)."""
+    for i, n in enumerate(n_vis):
+        g = idx_gpu[i]
+        K = min(k, n)
+        assert (g[K:] == -1).all(), f"row {i}: padding"
+        sel = g[:K]
+        assert (sel >= 0).all() and (sel < n).all(), f"row {i}: out of range"
+        assert (np.diff(sel) > 0).all(), f"row {i}: not strictly ascending"
+        r = scores_ref[i, :n]
+        order = np.lexsort((np.arange(n), -r))
+        kth = r[order[K - 1]]
+        band = SET_TOL_REL * np.max(np.abs(r))
+        ref_set = set(order[:K].tolist())
+        diff = ref_set.symmetric_difference(sel.tolist())
+        for s in diff:
+            assert abs(r[s] - kth) <= band, f"row {i}: position {s} differs with score gap {abs(r[s]-kth):.3e}"

@@ -1,0 +1,222 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Sizes span several 128-key tiles with ragged tails, every indexer schedule
+(1, 4 and 8 queries per tile; split and wave sweeps), rows shorter and longer
+than topk, ties, signed zeros, padded index lists and shared caches.
+"""
+import os
+import zlib
+
+import numpy as np
+import pytest
+
+import oracle
+from indexer_selected_sparse_dsa_b200 import binding as B
+from indexer_selected_sparse_dsa_b200 import workloads as wl
+
+from gpu_util import (SCALE, assert_attention_close, assert_scores_close, assert_selection_ok, gpu_attention,
+                      gpu_forward, gpu_scores, gpu_topk, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _lib():
+    from indexer_selected_sparse_dsa_b200 import build
+    build.build()
+    B.lib()
+
+
+# ---------------------------------------------------------------------------- indexer
+
+INDEXER_CASES = {
+    # name: (seq_lens, queries)
+    "one_row_ragged": ([700], [(0, 700)]),
+    "shared_cache_4": ([1000], [(0, 1000), (0, 999), (0, 640), (0, 1)]),
+    "mixed_sequences": ([300, 129, 1000], [(0, 300), (1, 129), (2, 1000), (2, 513), (0, 17), (2, 1000), (1, 1)]),
+    "causal_prefill": ([600], [(0, t + 1) for t in range(600)]),
+    "many_decode_rows": ([257] * 40, [(b, 257 - (b % 3)) for b in range(40)]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(INDEXER_CASES))
+@pytest.mark.parametrize("sweep", ["split", "wave"])
+def test_indexer_scores_match_oracle(name, sweep, monkeypatch):
+    monkeypatch.setenv("DSA_INDEXER_SWEEP", sweep)
+    seq_lens, queries = INDEXER_CASES[name]
+    c = wl.make_case_numpy(seq_lens, queries, seed=zlib.crc32(name.encode()) % 1000, n_plant=4)
+    ld = (max(c.n_vis) + 3) // 4 * 4 + 4
+    ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=ld)
+    got = gpu_scores(to_dev(c), ld).cpu().numpy()
+    assert_scores_close(got, ref, c.n_vis)
+    for i, n in enumerate(c.n_vis):     # columns past n_vis are not written
+        assert np.isnan(got[i, n:]).all(), f"row {i} wrote past n_vis"
+
+
+@pytest.mark.parametrize("qmax", ["1", "4", "8"])
+def test_indexer_every_tile_width(qmax, monkeypatch):
+    monkeypatch.setenv("DSA_INDEXER_QMAX", qmax)
+    c = wl.make_case_numpy([900, 400], [(0, 900), (0, 899), (0, 777), (1, 400), (1, 385), (0, 5)], seed=31, n_plant=4)
+    ld = 904
+    ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=ld)
+    got = gpu_scores(to_dev(c), ld).cpu().numpy()
+    assert_scores_close(got, ref, c.n_vis)
+
+
+def test_indexer_bad_row_is_skipped_and_reported():
+    import torch
+    c = wl.make_case_numpy([300], [(0, 300), (0, 200)], seed=3, n_plant=0)
+    d = to_dev(c)
+    d["n_vis"][1] = 0            # invalid: a query always sees itself
+    ld = 300
+    scores = torch.full((2, ld), float("nan"), device="cuda")
+    ws = B.workspace(B.DSA_OP_INDEXER, 2, ld, 0)
+    B.dsa_indexer_scores(d["q_I"], d["w"], d["k_I"], d["kv_start"], d["n_vis"], scores, ws)
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_sync_status()
+    assert e.value.code == B.DSA_ERR_BAD_ROW
+    s = scores.cpu().numpy()
+    ref = oracle.indexer_scores(c.q_I[:1], c.w[:1], c.k_I, c.kv_start[:1], c.n_vis[:1], score_ld=ld)
+    assert_scores_close(s[:1], ref, c.n_vis[:1])
+    assert np.isnan(s[1]).all()
+    B.dsa_sync_status()         # the status word was cleared
+
+
+# ---------------------------------------------------------------------------- top-k
+
+def _topk_case(kind, n, seed):
+    r = np.random.default_rng(seed)
+    if kind == "normal":
+        return r.standard_normal(n).astype(np.float32)
+    if kind == "ties":
+        return r.integers(-4, 5, size=n).astype(np.float32)
+    if kind == "equal":
+        return np.full(n, 0.75, np.float32)
+    if kind == "zeros":
+        z = np.zeros(n, np.float32)
+        z[r.random(n) < 0.5] = -0.0
+        z[r.random(n) < 0.1] = 1.0
+        return z
+    if kind == "wide":
+        return (r.standard_normal(n) * np.exp(r.uniform(-30, 30, n))).astype(np.float32)
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "wide"])
+@pytest.mark.parametrize("k", [1, 7, 2048])
+def test_topk_bit_exact(kind, k):
+    lens = [1, 5, k - 1 if k > 1 else 1, k, k + 1, 2047, 2049, 5000, 20000]
+    ld = (max(lens) + 3) // 4 * 4
+    S = np.full((len(lens), ld), np.nan, np.float32)
+    for i, n in enumerate(lens):
+        S[i, :n] = _topk_case(kind, n, seed=i * 7 + k)
+    n_vis = np.array(lens, np.int32)
+    ref = oracle.topk(S.astype(np.float64), n_vis, k)   # the same fp32 values, compared exactly
+    got = gpu_topk(S, n_vis, k)
+    for i in range(len(lens)):
+        assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
+
+
+def test_topk_long_row_exact():
+    n, k = 131072, 2048
+    S = _topk_case("normal", n, 5)[None]
+    ref = oracle.topk(S.astype(np.float64), np.array([n], np.int32), k)
+    assert np.array_equal(gpu_topk(S, [n], k), ref)
+
+
+# ---------------------------------------------------------------------------- attention
+
+def _attention_case(seed, L=3000, T=5, k=2048, pad=(0, 100, 1900, 2047, 0)):
+    c = wl.make_case_numpy([L], [(0, L)] * T, seed=seed, n_plant=0)
+    r = np.random.default_rng(seed)
+    idx = np.full((T, k), -1, np.int32)
+    for i in range(T):
+        m = k - pad[i % len(pad)]
+        idx[i, :m] = np.sort(r.choice(L, m, replace=False))
+    return c, idx
+
+
+def test_attention_matches_oracle_on_given_indices():
+    c, idx = _attention_case(41)
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+
+
+def test_attention_ragged_topk_and_gaps():
+    # topk not a multiple of 128, -1 holes inside the list, unsorted entries
+    c = wl.make_case_numpy([800], [(0, 800)] * 3, seed=43, n_plant=0)
+    r = np.random.default_rng(43)
+    k = 300
+    idx = r.choice(800, size=(3, k)).astype(np.int32)
+    idx[0, ::7] = -1
+    idx[1, :] = -1
+    idx[1, 5] = 123                     # single key: o = c_kv[123]
+    idx[2, 150:] = -1
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+
+
+def test_attention_empty_row_and_large_logits():
+    c = wl.make_case_numpy([500], [(0, 500)] * 2, seed=44, n_plant=0)
+    qf = wl.bf16_to_f32(c.q) * 8.0     # logits up to ~ +-40: exercises the lazy rescale
+    c.q = wl.bf16_from_f32(qf)
+    idx = np.full((2, 512), -1, np.int32)
+    idx[0] = np.arange(500, dtype=np.int32).tolist() + [-1] * 12
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+    assert (o[1] == 0).all() and np.isneginf(lse[1]).all()
+
+
+def test_attention_per_row_cache_offsets():
+    c = wl.make_case_numpy([700, 900, 300], [(0, 700), (1, 900), (2, 300), (1, 450)], seed=45, n_plant=0)
+    r = np.random.default_rng(45)
+    k = 640
+    idx = np.full((4, k), -1, np.int32)
+    for i, n in enumerate(c.n_vis):
+        m = min(k, int(n))
+        idx[i, :m] = np.sort(r.choice(int(n), m, replace=False))
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+
+
+# ---------------------------------------------------------------------------- whole step
+
+def _forward_check(c, k=2048):
+    d = to_dev(c)
+    maxn = int(max(c.n_vis))
+    o, lse, idx = gpu_forward(d, maxn, k)
+    S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=maxn)
+    assert_selection_ok(idx, S_ref, c.n_vis, k)
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)   # on the GPU's index set
+    assert_attention_close(o, lse, o_ref, lse_ref)
+    for i in range(c.T):                          # planted positions are recalled
+        p = c.plants[i][c.plants[i] >= 0]
+        assert np.isin(p, idx[i]).all(), f"row {i}: planted position dropped"
+    return idx
+
+
+def test_forward_decode_shared_cache_scaled():
+    _forward_check(wl.make_workload_numpy(0, scale=4))       # 4 queries over 8192 shared rows
+
+
+def test_forward_decode_per_sequence_scaled():
+    c = wl.make_case_numpy([6000] * 6, [(b, 6000 - 7 * b) for b in range(6)], seed=1)
+    _forward_check(c)
+
+
+def test_forward_causal_prefill_short_rows():
+    # rows t < topk keep every prior position; later rows select
+    c = wl.make_case_numpy([2600], [(0, t + 1) for t in range(0, 2600, 37)] + [(0, 2048), (0, 2049), (0, 2600)],
+                           seed=2)
+    idx = _forward_check(c)
+    for i, n in enumerate(c.n_vis):
+        if n <= 2048:
+            assert idx[i, :n].tolist() == list(range(n))
+
+
+def test_forward_ragged_decode_scaled():
+    _forward_check(wl.make_workload_numpy(3, scale=32))
