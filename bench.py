@@ -1,0 +1,484 @@
+"""Benchmark of the DSA sparse-attention step (indexer -> top-k -> sparse MLA).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config C] [--scale S] [--skip-cpu] [--skip-e2e]
+
+One step = one dsa_forward over one batch of the workload (every query row:
+indexer over its causal context, exact top-2048, sparse latent MLA).  The
+default workload is batch-64 decode at 131072 context per sequence.  Inputs
+are synthetic (seeded) and resident in HBM; the per-step working set (about
+2.3 GB) is far larger than the 126 MB L2, so no L2 flush is needed between
+steps.  Under torchrun every rank runs its own batch (weak scaling; the
+path has no data exchange between rows).  Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload shape
+(rank 0 only; bounded samples of query rows per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from indexer_selected_sparse_dsa_b200 import workloads as wl  # noqa: E402
+
+METRIC_DECODE = "decode tokens/s"
+METRIC_PREFILL = "prefill query-tokens/s"
+TOPK = wl.TOPK
+
+
+def metric_for(cfg):
+    return METRIC_DECODE if wl.WORKLOADS[cfg]["kind"] == "decode" else METRIC_PREFILL
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- work model
+
+def work_model(n_vis: np.ndarray, topk: int = TOPK):
+    """Algorithmic bytes and flops of one step, per component (the units the
+    roofline fractions use).  n_vis: visible positions of each query row."""
+    n = n_vis.astype(np.float64)
+    sel = np.minimum(n, topk)
+    q_idx = 32 * 128 * 2 + 32 * 2                      # q_I + w per row
+    idx_bytes = 256 * n + 4 * n + q_idx                 # keys read, scores written
+    idx_flops = 2 * 32 * 128 * n                        # 32-head form
+    topk_bytes = 4 * n + 4 * topk                       # scores read, indices written
+    att_bytes = 1152 * sel + 64 * 576 * 2 + 64 * 512 * 4 + 64 * 4 + 4 * topk
+    att_flops = 2 * 64 * sel * (576 + 512)
+    step_bytes = 256 * n + q_idx + 1152 * sel + 64 * 576 * 2 + 64 * 512 * 4 + 64 * 4
+    return dict(indexer_bytes=idx_bytes.sum(), indexer_flops=idx_flops.sum(), topk_bytes=topk_bytes.sum(),
+                attention_bytes=att_bytes.sum(), attention_flops=att_flops.sum(), step_bytes=step_bytes.sum(),
+                step_flops=(idx_flops + att_flops).sum())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None, interval_ms: int = 50):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", str(interval_ms)]
+        if bus_id:
+            cmd += ["-i", bus_id]
+        try:
+            self.p = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+        self.lines: list[str] = []
+
+    def stop(self):
+        if self.p is None:
+            return
+        time.sleep(0.12)
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+            out, _ = self.p.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bus_id_of(dev):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- profiles
+
+def lib_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "indexer_selected_sparse_dsa_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel sources (same source hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d[f"{kernel}/{workload}"]
+        if e.get("source_hash") == lib_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+    from indexer_selected_sparse_dsa_b200 import binding as B
+    from indexer_selected_sparse_dsa_b200 import build
+
+    build.build()
+    B.lib()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    cfg, scale = args.config, args.scale
+    c = wl.make_workload_torch(cfg, dev, scale=scale, seed=cfg + 7919 * rank)
+    T = c.T
+    n_vis_h = c.n_vis.cpu().numpy()
+    max_n = int(n_vis_h.max())
+    k = TOPK
+    o = torch.empty((T, 64, 512), dtype=torch.float32, device=dev)
+    lse = torch.empty((T, 64), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    ws = B.workspace(B.DSA_OP_FORWARD, T, max_n, k, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        B.dsa_forward(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, max_n, k, wl.SCALE, o, lse, idx, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    B.dsa_sync_status(stream)
+
+    # ---- timed region: exactly K steps of dsa_forward
+    sampler = ClockSampler(bus_id_of(dev))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    B.dsa_sync_status(stream)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    sampler.stop()
+    clocks = sampler.summary()
+    if clocks is None or clocks["samples"] < 3:
+        # timed region shorter than the sampling interval: sample an equal-load loop
+        s2 = ClockSampler(bus_id_of(dev))
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize(dev)
+        s2.stop()
+        clocks = s2.summary()
+        if clocks is not None:
+            clocks["note"] = "sampled during an equal-load loop right after the timed region (timed region too short)"
+    ms_step = ms / args.steps
+
+    # ---- per-kernel breakdown: the same kernels through the component entry points
+    nb = max(3, min(args.steps, 50))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
+    plan_ws = B.workspace(B.DSA_OP_INDEXER, T, max_n, k, device=dev)
+    ld = (max_n + 3) // 4 * 4
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        e[0].record(stream)
+        B.dsa_indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, scores, plan_ws, stream)
+        e[1].record(stream)
+        B.dsa_topk(scores, c.n_vis, k, idx, stream)
+        e[2].record(stream)
+        B.dsa_sparse_mla_attn(c.q, c.kv, c.kv_start, idx, wl.SCALE, o, lse, None, stream)
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    B.dsa_sync_status(stream)
+    t_idx = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_topk = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    t_att = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    wm = work_model(n_vis_h)
+    pk = peaks()
+    workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
+    idx_gbs = wm["indexer_bytes"] / (t_idx * 1e-3) / 1e9
+    roofline = {"kernel": "indexer (dsa_indexer_scores: plan + tcgen05 kernel)", "bound": "hbm",
+                "achieved": round(idx_gbs, 1), "peak": pk["hbm"], "unit": "GB/s",
+                "frac": round(idx_gbs / pk["hbm"], 4), "peak_source": pk["source"],
+                "traffic": profiled_traffic("indexer", workload),
+                "algorithmic_bytes_per_launch": float(wm["indexer_bytes"]),
+                "launch_ms": round(t_idx, 4)}
+    step_gbs = wm["step_bytes"] / (ms_step * 1e-3) / 1e9
+    kernels = {
+        "indexer": {"ms": round(t_idx, 4), "GB/s": round(idx_gbs, 1),
+                    "TFLOP/s": round(wm["indexer_flops"] / (t_idx * 1e-3) / 1e12, 1)},
+        "topk": {"ms": round(t_topk, 4), "GB/s": round(wm["topk_bytes"] / (t_topk * 1e-3) / 1e9, 1)},
+        "sparse_mla": {"ms": round(t_att, 4), "GB/s": round(wm["attention_bytes"] / (t_att * 1e-3) / 1e9, 1),
+                       "TFLOP/s": round(wm["attention_flops"] / (t_att * 1e-3) / 1e12, 1)},
+    }
+
+    # ---- end to end through dsa_forward with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        e2e = run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist)
+        if e2e is not None:
+            e2e["value"] = round(T * world / (e2e.pop("ms_per_step") * 1e-3), 1)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = cpu_baseline(c, o, lse, idx, args)
+
+    value = T * world / (ms_step * 1e-3)
+    out = {
+        "metric": metric_for(cfg), "value": round(value, 1),
+        "unit": "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload, "batch_rows": T, "max_context": max_n, "topk": k,
+                   "indexer_heads": 32, "indexer_dim": 128, "mla_heads": 64, "kv_lora_rank": 512, "rope_dim": 64,
+                   "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+        "roofline": roofline,
+        "step_roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": pk["hbm"], "unit": "GB/s",
+                          "frac": round(step_gbs / pk["hbm"], 4),
+                          "algorithmic_bytes_per_step": float(wm["step_bytes"])},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
+    """dsa_forward with the step's inputs copied in from pinned host memory and
+    its result copied out, every step.  The cache stays resident (it is state
+    that persists across decode steps); the rows this step appends to it (the
+    new token's k_I and latent row of each sequence) are part of the copy-in."""
+    import torch
+    from indexer_selected_sparse_dsa_b200 import binding as B
+    T = c.T
+    new_rows = (c.kv_start + c.n_vis.to(torch.int64) - 1)
+    h = {
+        "q_I": c.q_I.cpu().pin_memory(), "w": c.w.cpu().pin_memory(), "q": c.q.cpu().pin_memory(),
+        "kv_start": c.kv_start.cpu().pin_memory(), "n_vis": c.n_vis.cpu().pin_memory(),
+        "k_new": c.k_I[new_rows].cpu().pin_memory(), "kv_new": c.kv[new_rows].cpu().pin_memory(),
+        "rows": new_rows.cpu().pin_memory(),
+    }
+    d = {kk: torch.empty_like(v, device=dev) for kk, v in h.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    bi = sum(v.numel() * v.element_size() for v in h.values())
+    bo = o_h.numel() * 4 + lse_h.numel() * 4
+
+    def step():
+        for kk in h:
+            d[kk].copy_(h[kk], non_blocking=True)
+        c.k_I.index_copy_(0, d["rows"], d["k_new"])
+        c.kv.index_copy_(0, d["rows"], d["kv_new"])
+        B.dsa_forward(d["q_I"], d["w"], c.k_I, d["q"], c.kv, d["kv_start"], d["n_vis"], max_n, k, wl.SCALE,
+                      o, lse, idx, ws, stream)
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    steps = args.steps
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    B.dsa_sync_status(stream)
+    return {"ms_per_step": ms / steps, "unit": "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s",
+            "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "api": "dsa_forward"}
+
+
+def cpu_baseline(c, o, lse, idx, args, budget_s: float = 15.0):
+    """The oracle, as it stands, on the host cores over a bounded sample of this
+    run's own query rows (their caches copied back); also reports how far the
+    GPU's outputs for those rows are from the oracle's."""
+    import torch
+    import oracle
+    from indexer_selected_sparse_dsa_b200.workloads import case_to_host  # noqa: F401
+    cores = os.cpu_count() or 1
+    T = c.T
+    rows_done, t_spent, maxerr = 0, 0.0, 0.0
+    order = list(range(T))
+    batch = min(cores, T)
+    while rows_done < T and t_spent < budget_s:
+        rows = order[rows_done:rows_done + batch]
+        # compact copies of just these rows' sequences
+        q_I = c.q_I[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        w = c.w[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        q = c.q[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        ks = c.kv_start[rows].cpu().numpy()
+        nv = c.n_vis[rows].cpu().numpy()
+        kI_parts, kv_parts, starts = [], [], []
+        off = 0
+        for s0, n in zip(ks, nv):
+            kI_parts.append(c.k_I[int(s0):int(s0) + int(n)].view(torch.int16).cpu().numpy().view(np.uint16))
+            kv_parts.append(c.kv[int(s0):int(s0) + int(n)].view(torch.int16).cpu().numpy().view(np.uint16))
+            starts.append(off)
+            off += int(n)
+        kI = np.concatenate(kI_parts)
+        kv = np.concatenate(kv_parts)
+        t0 = time.perf_counter()
+        o_ref, lse_ref, idx_ref = oracle.forward(q_I, w, kI, q, kv, np.array(starts, np.int64), nv, TOPK, wl.SCALE,
+                                                 nthreads=cores)
+        t_spent += time.perf_counter() - t0
+        rows_done += len(rows)
+        g = o[rows].cpu().numpy().astype(np.float64)
+        maxerr = max(maxerr, float(np.max(np.abs(g - o_ref))))
+    unit = "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s"
+    return {"value": round(rows_done / t_spent, 3), "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{rows_done} of {T} query rows of this run (full context each), fp64 C++ oracle, {t_spent:.1f} s",
+            "gpu_vs_oracle_max_abs_on_sample": maxerr}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    cores = os.cpu_count() or 1
+    cfg, scale = args.config, args.scale
+    seq_lens, queries, _kind = wl.workload_layout(cfg, scale)
+    # a bounded host-side replica of the workload: the first few sequences / rows
+    if wl.WORKLOADS[cfg]["kind"] == "decode":
+        nseq = min(len(seq_lens), max(1, min(cores, 8)))
+        c = wl.make_case_numpy(seq_lens[:nseq], [q for q in queries if q[0] < nseq], seed=cfg)
+    else:
+        nq = min(len(queries), max(1, min(cores, 8)))
+        c = wl.make_case_numpy(seq_lens, queries[-nq:], seed=cfg)
+    rows_per_step = min(c.T, cores)
+    budget = 150.0
+    times, rows_total = [], 0
+    t_start = time.perf_counter()
+    steps_done = 0
+    r = 0
+    for s in range(args.warmup + args.steps):
+        sel = [(r + j) % c.T for j in range(rows_per_step)]
+        r += rows_per_step
+        t0 = time.perf_counter()
+        oracle.forward(c.q_I[sel], c.w[sel], c.k_I, c.q[sel], c.kv, c.kv_start[sel], c.n_vis[sel], TOPK, wl.SCALE,
+                       nthreads=cores)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            rows_total += len(sel)
+            steps_done += 1
+        if time.perf_counter() - t_start > budget and steps_done >= 1:
+            break
+    tot = sum(times)
+    value = rows_total / tot
+    unit = "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s"
+    workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
+    out = {"impl": "reference", "metric": metric_for(cfg), "value": round(value, 4), "unit": unit, "n_gpus": world,
+           "steps": steps_done, "steps_requested": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * tot / max(steps_done, 1), 2), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": workload, "batch_rows": len(queries), "max_context": int(max(q[1] for q in queries)),
+                      "topk": TOPK, "rows_per_step": rows_per_step},
+           "cpu_baseline": {"kind": "oracle", "cores": cores, "value": round(value, 4), "unit": unit,
+                            "sample": f"{rows_per_step} query rows per step (full context each) of the workload, "
+                                      f"fp64 C++ oracle, {steps_done} steps in {tot:.1f} s"},
+           "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1, help="workload: 0..4 (default 1: decode b64 x 128K)")
+    ap.add_argument("--scale", type=int, default=1, help="shrink contexts by this factor (small captures)")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
