@@ -163,6 +163,34 @@ DSA_API int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* 
                 dsa_stream_t stream);
 
 /*
+ * dsa_indexer_scores without a workspace argument: the same scores, for
+ * callers that cannot allocate device memory.  There is no counterpart on
+ * the pages; this is a library-interface addition.
+ *
+ * Who needs it: code that runs inside a host framework which owns every
+ * byte of device memory and allows no allocation once it has started (a
+ * serving engine with a memory pool planned at start-up, a plug-in whose
+ * host interface hands it tensors but no allocator).  For such callers
+ * cudaMalloc is either unavailable or would synchronise the device in the
+ * middle of a step.
+ *
+ * Scratch: the per-call query-tile plan lives in a fixed array in the
+ * library's own device memory (DSA_NOALLOC_MAX_ROWS rows, about 256 KB),
+ * which every GPU that loads the library holds until the process exits.
+ * T above DSA_NOALLOC_MAX_ROWS is rejected with DSA_ERR_INVALID_ARG.
+ * The first call on a device looks up that array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array and each call overwrites what the previous
+ * one left there, so calls whose execution overlaps on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ * Arguments and errors otherwise as dsa_indexer_scores.
+ */
+#define DSA_NOALLOC_MAX_ROWS 8192
+DSA_API int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I,
+                                       int64_t cache_rows, const int64_t* kv_start, const int32_t* n_vis, int T,
+                                       float* scores, int64_t score_ld, dsa_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_BAD_ROW or
  * DSA_ERR_CUDA (a sticky CUDA error).

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_UNSUPPORTED, DSA_ERR_BAD_ROW = range(7)
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD = range(4)
 INDEX_HEADS, INDEX_DIM, HEADS, LATENT, ROPE, ROW, MAX_TOPK = 32, 128, 64, 512, 64, 576, 2048
+NOALLOC_MAX_ROWS = 8192
 
 _STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_WORKSPACE", 3: "DSA_ERR_CUDA",
                  4: "DSA_ERR_TIMEOUT", 5: "DSA_ERR_UNSUPPORTED", 6: "DSA_ERR_BAD_ROW"}
@@ -46,6 +47,8 @@ def lib():
         L.dsa_sparse_mla_attn.argtypes = [P, P, I64, P, P, I, I, F, P, P, P, SZ, P]
         L.dsa_forward.argtypes = [P, P, P, P, P, I64, P, P, I, I64, I, F, P, P, P, P, SZ, P]
         L.dsa_sync_status.argtypes = [P]
+        L.dsa_indexer_scores_noalloc.argtypes = [P, P, P, I64, P, P, I, P, I64, P]
+        L.dsa_indexer_scores_noalloc.restype = I
         L.dsa_last_error_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I
         for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_sync_status"):
@@ -102,6 +105,22 @@ def dsa_indexer_scores(q_I, w, k_I, kv_start, n_vis, scores, ws, stream=None):
     _need(ws, torch.uint8, None, "ws")
     _check(lib().dsa_indexer_scores(_ptr(q_I), _ptr(w), _ptr(k_I), k_I.shape[0], _ptr(kv_start), _ptr(n_vis), T,
                                     _ptr(scores), scores.shape[1], _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def dsa_indexer_scores_noalloc(q_I, w, k_I, kv_start, n_vis, scores, stream=None):
+    """dsa_indexer_scores for callers that cannot allocate: no workspace; the
+    library keeps the plan in its own fixed device array (at most
+    NOALLOC_MAX_ROWS rows; calls must not overlap on the GPU)."""
+    import torch
+    T = n_vis.shape[0]
+    _need(q_I, torch.bfloat16, (T, INDEX_HEADS, INDEX_DIM), "q_I")
+    _need(w, torch.bfloat16, (T, INDEX_HEADS), "w")
+    _need(k_I, torch.bfloat16, None, "k_I")
+    _need(kv_start, torch.int64, (T,), "kv_start")
+    _need(n_vis, torch.int32, (T,), "n_vis")
+    _need(scores, torch.float32, None, "scores")
+    _check(lib().dsa_indexer_scores_noalloc(_ptr(q_I), _ptr(w), _ptr(k_I), k_I.shape[0], _ptr(kv_start),
+                                            _ptr(n_vis), T, _ptr(scores), scores.shape[1], _stream(stream)))
 
 
 def dsa_topk(scores, n_vis, topk, idx, stream=None):

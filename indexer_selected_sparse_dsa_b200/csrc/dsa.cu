@@ -19,6 +19,14 @@
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
+// Scratch of dsa_indexer_scores_noalloc: the query-tile plan for up to
+// DSA_NOALLOC_MAX_ROWS rows (about 256 KB).  Every device that loads this
+// library holds its own copy until the process exits; all calls of that entry
+// point on a device share it.
+static constexpr size_t kNoAllocPlanBytes =
+    sizeof(dsa::PlanHeader) + sizeof(dsa::PlanTile) * size_t(DSA_NOALLOC_MAX_ROWS);
+static __device__ __align__(256) unsigned char g_noalloc_plan[kNoAllocPlanBytes];
+
 namespace {
 
 thread_local std::string t_err;
@@ -47,6 +55,7 @@ struct DeviceState {
   bool supported = false;
   bool prepared = false;
   int sm_count = 0;
+  void* noalloc_plan = nullptr;  // device address of g_noalloc_plan on this device
 };
 constexpr int kMaxDevices = 64;
 DeviceState g_dev[kMaxDevices];
@@ -309,6 +318,36 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   e = dsa::launch_sparse_mla(p);
   if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
   return DSA_OK;
+}
+
+int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                               const int64_t* kv_start, const int32_t* n_vis, int T, float* scores, int64_t score_ld,
+                               dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (T > DSA_NOALLOC_MAX_ROWS)
+    return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_scores_noalloc handles at most %d query rows (got %d)",
+                DSA_NOALLOC_MAX_ROWS, T);
+  if (T == 0) return DSA_OK;
+  if (!q_I || !w || !k_I || !n_vis || !scores) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_I, 16) || !aligned(w, 16) || !aligned(k_I, 16) || !aligned(scores, 16) || !aligned(n_vis, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q_I, w, k_I, scores must be 16-byte aligned and n_vis 4-byte aligned");
+  if (score_ld < 4 || score_ld % 4 != 0) return fail(DSA_ERR_INVALID_ARG, "score_ld must be a positive multiple of 4");
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  if (!dev->noalloc_plan) {
+    // Once per device, with that device current: the host-side name of the array
+    // is not a device address, so ask the runtime for this device's copy.
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_plan);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(plan scratch)");
+    dev->noalloc_plan = ptr;
+  }
+  // The plan kernel rewrites every header and tile entry it uses, so the array
+  // needs no clearing between calls.
+  return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, score_ld, dev->noalloc_plan, stream,
+                     dev->sm_count);
 }
 
 int dsa_sync_status(dsa_stream_t stream) {
