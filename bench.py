@@ -154,6 +154,28 @@ def profiled_traffic(kernel: str, workload: str):
     return None
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def reduce_max_ms(ms: float, dist, device) -> float:
+    """Max of a per-rank time over all ranks (every rank calls this)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(rows_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Units of all ranks per second, timed by the slowest rank."""
+    return rows_per_rank * world / (ms_per_step * 1e-3)
+
+
+def rank_seed(cfg: int, rank: int) -> int:
+    """Each rank draws its own replica batch (weak scaling)."""
+    return cfg + 7919 * rank
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, dist):
@@ -166,7 +188,7 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     cfg, scale = args.config, args.scale
-    c = wl.make_workload_torch(cfg, dev, scale=scale, seed=cfg + 7919 * rank)
+    c = wl.make_workload_torch(cfg, dev, scale=scale, seed=rank_seed(cfg, rank))
     T = c.T
     n_vis_h = c.n_vis.cpu().numpy()
     max_n = int(n_vis_h.max())
@@ -199,10 +221,7 @@ def run_ours(args, rank, world, dist):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     B.dsa_sync_status(stream)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max_ms(ms, dist, dev)
     sampler.stop()
     clocks = sampler.summary()
     if clocks is None or clocks["samples"] < 3:
@@ -264,13 +283,13 @@ def run_ours(args, rank, world, dist):
     if not args.skip_e2e:
         e2e = run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist)
         if e2e is not None:
-            e2e["value"] = round(T * world / (e2e.pop("ms_per_step") * 1e-3), 1)
+            e2e["value"] = round(whole_job_rate(T, world, e2e.pop("ms_per_step")), 1)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
         cpu = cpu_baseline(c, o, lse, idx, args)
 
-    value = T * world / (ms_step * 1e-3)
+    value = whole_job_rate(T, world, ms_step)
     out = {
         "metric": metric_for(cfg), "value": round(value, 1),
         "unit": "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s",
@@ -339,11 +358,7 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max_ms(e0.elapsed_time(e1), dist, dev)
     B.dsa_sync_status(stream)
     return {"ms_per_step": ms / steps, "unit": "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s",
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "api": "dsa_forward"}

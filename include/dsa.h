@@ -3,14 +3,14 @@
  * lightning indexer -> per-row top-k -> sparse MLA attention in latent form.
  *
  * What the step computes (pages on the method; page title and section):
- *  - "GLM 5 DSV3.2 DSA MoE configuration", section 2.2: a lightweight
+ *  - "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2: a lightweight
  *    indexer scores every query against all of its history and is used only
  *    to rank; a top-k selector keeps index_topk = 2048 positions; real MLA
  *    attention runs over those positions only.
  *  - same page, section 2.1 (config table): index_n_heads 32,
  *    index_head_dim 128, num_attention_heads 64, kv_lora_rank 512,
  *    qk_rope_head_dim 64, qk_head_dim 256, index_topk 2048.
- *  - "DSA + IndexShare explainer", section "DSA full flow": indexer over all
+ *  - "From a trillion dot products to two thousand: how DSA breaks N^2", section "DSA full flow": indexer over all
  *    history -> top-2048 -> softmax over the 2048 and the value mix; the KV
  *    cache keeps unselected positions for other queries.
  *  The score and attention formulas (stated on each function) are the
@@ -88,9 +88,9 @@ enum dsa_op {
 DSA_API size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk);
 
 /*
- * Lightning-indexer scores ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2;
- * "DSA + IndexShare explainer", section "lightning indexer: low-dimensional
- * dot products"):
+ * Lightning-indexer scores ("2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2;
+ * "From a trillion dot products to two thousand: how DSA breaks N^2", section "how is the coarse screen fast? low
+ * dimensions"):
  *     scores[i, s] = sum_{h<32} w[i,h] * (q_I[i,h,:] . k_I[kv_start[i]+s, :])
  * for 0 <= s < n_vis[i], computed from bf16 inputs with fp32 accumulation on
  * the tensor cores.  Columns s >= n_vis[i] of the row are not written.
@@ -108,8 +108,8 @@ DSA_API int dsa_indexer_scores(const dsa_bf16* q_I, const dsa_bf16* w, const dsa
                        void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /*
- * Top-k selector ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2: keep the
- * index_topk highest-scoring positions; "DSA + IndexShare explainer",
+ * Top-k selector ("2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2: keep the
+ * index_topk highest-scoring positions; "From a trillion dot products to two thousand: how DSA breaks N^2",
  * index_topk: 2048).  For row i keeps K = min(topk, n_vis[i]) positions of
  * scores[i, 0:n_vis[i]] under the total order (score descending, position
  * ascending: ties go to the lower position; -0.0 equals +0.0), writes them in
@@ -125,7 +125,7 @@ DSA_API int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis
 
 /*
  * Sparse MLA attention in latent (absorbed) form over the selected rows
- * ("DSA + IndexShare explainer", "DSA full flow": full Q.K, softmax and the
+ * ("From a trillion dot products to two thousand: how DSA breaks N^2", "DSA full flow": full Q.K, softmax and the
  * value mix over the selected 2048 only; config table: qk_head_dim 256 so the
  * softmax scale is 1/sqrt(256)).  For row i, head h and the valid entries
  * s_j = idx[i,j] >= 0:

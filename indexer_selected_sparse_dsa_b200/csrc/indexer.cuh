@@ -2,7 +2,7 @@
 //
 //   scores[i, s] = sum_{h<32} w[i,h] * (q_I[i,h,:] . k_I[kv_start[i]+s, :])
 //
-// ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2: a light scorer of every
+// ("2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2: a light scorer of every
 // query against all history, 32 heads x 128 dims; the per-head weighting and
 // head sum are the problem statement's.)
 //

@@ -3,8 +3,8 @@
 //   S[h,j]   = scale * (q_lat[h] . c_kv[s_j] + q_rope[h] . k_rope[s_j])
 //   o_lat[h] = sum_j softmax_j(S[h,:]) c_kv[s_j],   lse[h] = log sum_j exp S[h,j]
 //
-// ("DSA + IndexShare explainer", "DSA full flow": full Q.K, softmax and the
-// value mix over the selected 2048 only; "GLM 5 DSV3.2 DSA MoE configuration",
+// ("From a trillion dot products to two thousand: how DSA breaks N^2", "DSA full flow": full Q.K, softmax and the
+// value mix over the selected 2048 only; "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2",
 // section 2.1: 64 heads, kv_lora_rank 512, rope 64, qk_head_dim 256.)
 //
 // One CTA per query row.  The selected 1152-byte rows are gathered 128 at a

@@ -1,6 +1,6 @@
 // Exact per-row top-k over materialised fp32 indexer scores.
 //
-// ("GLM 5 DSV3.2 DSA MoE configuration", section 2.2: keep the index_topk
+// ("2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2: keep the index_topk
 // highest-scoring positions; ties go to the lower position, the kept
 // positions are written in ascending order and padded with -1.)
 //

@@ -6,7 +6,7 @@ the CUDA path and the fp64 oracle consume the exact bf16 bit patterns it
 produces, so the two sides share inputs and nothing else.
 
 Shapes follow the GLM-5 / DeepSeek-V3.2 attention config table (page
-"GLM 5 DSV3.2 DSA MoE configuration", section 2.1): 32 indexer heads of dim
+"2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.1): 32 indexer heads of dim
 128 (section 2.2), 64 MLA heads, kv_lora_rank 512, qk_rope_head_dim 64,
 index_topk 2048.  The value laws are:
 

@@ -6,13 +6,13 @@
 // path; the fixed dimensions below are restated here on purpose.
 //
 // Sources (pages on the method; the page title and section are cited):
-//  * "GLM 5 DSV3.2 DSA MoE configuration" (nlpx.cn), section 2.1 config table:
+//  * "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2" (nlpx.cn), section 2.1 config table:
 //    index_n_heads 32, index_head_dim 128, num_attention_heads 64,
 //    kv_lora_rank 512, qk_rope_head_dim 64, qk_head_dim 256, index_topk 2048.
 //  * same page, section 2.2: the lightning indexer scores each query against
 //    every history position, is used only for ranking, and a top-k selector
 //    keeps the index_topk best positions for the real attention.
-//  * "DSA + IndexShare explainer" (clawlihai.cn), "DSA full flow": stage one is
+//  * "From a trillion dot products to two thousand: how DSA breaks N^2" (clawlihai.cn), "DSA full flow": stage one is
 //    the low-dimensional indexer dot product over all history and a top-2048;
 //    stage two is full Q.K, softmax and the V mix over those 2048 only.
 //  * The score form I[t,s] = sum_h w[t,h] * (q_I[t,h] . k_I[s]) with one key per

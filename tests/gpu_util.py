@@ -110,3 +110,27 @@ def assert_selection_ok(idx_gpu, scores_ref, n_vis, k):
         diff = ref_set.symmetric_difference(sel.tolist())
         for s in diff:
             assert abs(r[s] - kth) <= band, f"row {i}: position {s} differs with score gap {abs(r[s]-kth):.3e}"
+
+
+def host_rows(c, rows):
+    """Compact host copies (uint16 bf16 bits) of some query rows of a torch case:
+    their query tensors and only their own visible cache prefixes, re-based so
+    row j's sequence starts at the returned kv_start[j]."""
+    import torch
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    ks = c.kv_start.cpu().numpy()
+    nv = c.n_vis.cpu().numpy()
+    kI, kv, starts = [], [], []
+    off = 0
+    for r in rows:
+        s0, n = int(ks[r]), int(nv[r])
+        kI.append(u16(c.k_I[s0:s0 + n]))
+        kv.append(u16(c.kv[s0:s0 + n]))
+        starts.append(off)
+        off += n
+    return dict(q_I=u16(c.q_I[rows]), w=u16(c.w[rows]), q=u16(c.q[rows]), k_I=np.concatenate(kI),
+                kv=np.concatenate(kv), kv_start=np.array(starts, np.int64), n_vis=nv[rows].astype(np.int32),
+                plants=c.plants[rows])

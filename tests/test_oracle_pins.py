@@ -3,9 +3,9 @@
 The pins are closed forms, algebraic identities that take a different route
 through the arithmetic, textbook routines from scipy, brute force on tiny
 inputs, and structural invariants stated on the pages:
-  * "GLM 5 DSV3.2 DSA MoE configuration", section 2.2 — the indexer only ranks,
+  * "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2 — the indexer only ranks,
     at most index_topk positions per query take part in attention;
-  * "DSA + IndexShare explainer", "DSA full flow" — indexer over all history,
+  * "From a trillion dot products to two thousand: how DSA breaks N^2", "DSA full flow" — indexer over all history,
     top-2048, then softmax and V mix over those only;
   * same page, on the kept KV cache — unselected positions stay available to
     other queries (a shared cache is read, never consumed).
