@@ -142,7 +142,11 @@ DSA_API int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis
  *  idx     [T,topk] int32: positions relative to kv_start, -1 = empty slot;
  *          entries with kv_start+idx >= cache_rows are skipped (status bit)
  *  o_lat   [T,64,512] fp32, 16-byte aligned; lse [T,64] fp32 or NULL
- *  ws      >= dsa_workspace_size(DSA_OP_SPARSE_MLA, T, 0, topk) bytes, 256-byte aligned
+ *  ws      dsa_workspace_size(DSA_OP_SPARSE_MLA, T, 0, topk) bytes, 256-byte
+ *          aligned, or NULL.  With few rows the selected positions of a row are
+ *          split over several CTAs whose fp32 partial results go to ws and are
+ *          merged by a second kernel; a NULL or smaller ws only reduces that
+ *          split (down to one CTA per row), never the result.
  */
 DSA_API int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
                         const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,

@@ -82,6 +82,7 @@ int current_device(DeviceState** out) {
   if (!d.prepared) {
     if ((e = dsa::prepare_indexer()) != cudaSuccess) return cuda_fail(e, "indexer smem opt-in");
     if ((e = dsa::prepare_sparse_mla()) != cudaSuccess) return cuda_fail(e, "sparse MLA smem opt-in");
+    if ((e = dsa::prepare_topk()) != cudaSuccess) return cuda_fail(e, "top-k smem opt-in");
     d.prepared = true;
   }
   *out = &d;
@@ -137,9 +138,11 @@ int64_t score_ld_for(int64_t max_n_vis) { return (max_n_vis + 3) / 4 * 4; }
 
 size_t ws_indexer(int T) { return align_up(dsa::indexer_plan_bytes(T), 256); }
 
+size_t ws_mla(int T, int topk) { return align_up(dsa::sparse_mla_part_bytes(T, dsa::sparse_mla_ws_splits(T, topk)), 256); }
+
 size_t ws_forward(int T, int64_t max_n_vis, int topk) {
   return ws_indexer(T) + align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256) +
-         align_up(size_t(T) * size_t(topk) * 4, 256);
+         align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
 }
 
 int pick_qmax(int T) {
@@ -157,6 +160,16 @@ int check_common_rows(int T, int64_t cache_rows, const void* kv_start) {
     return fail(DSA_ERR_INVALID_ARG, "cache_rows must lie in [1, 2^31-1] (got %lld)", (long long)cache_rows);
   if (T > 0 && !kv_start) return fail(DSA_ERR_INVALID_ARG, "kv_start is NULL");
   if (!aligned(kv_start, 8)) return fail(DSA_ERR_INVALID_ARG, "kv_start must be 8-byte aligned");
+  return DSA_OK;
+}
+
+int run_sparse_mla(const dsa::MlaLaunch& p) {
+  if (int64_t(p.T) * DSA_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
+  CUtensorMap tq;
+  int rc = make_tmap_bf16(&tq, p.q, DSA_ROW, uint64_t(p.T) * DSA_HEADS, 64);
+  if (rc) return rc;
+  cudaError_t e = dsa::launch_sparse_mla(p, tq);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
   return DSA_OK;
 }
 
@@ -212,7 +225,7 @@ size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
   switch (op) {
     case DSA_OP_INDEXER: return ws_indexer(T);
     case DSA_OP_TOPK: return 0;
-    case DSA_OP_SPARSE_MLA: return 0;
+    case DSA_OP_SPARSE_MLA: return ws_mla(T, topk);
     case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
     default: return 0;
   }
@@ -262,8 +275,6 @@ int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_row
                         const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,
                         size_t ws_bytes, dsa_stream_t stream) {
   t_err.clear();
-  (void)ws;
-  (void)ws_bytes;
   int rc = check_common_rows(T, cache_rows, kv_start);
   if (rc) return rc;
   if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
@@ -272,12 +283,13 @@ int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_row
   if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o_lat, 16) || !aligned(idx, 4) || !aligned(lse, 4))
     return fail(DSA_ERR_INVALID_ARG, "q, kv, o_lat must be 16-byte aligned; idx, lse 4-byte aligned");
   if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (ws && !aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
   DeviceState* dev = nullptr;
   if ((rc = current_device(&dev))) return rc;
-  dsa::MlaLaunch p{q, kv, cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, wait_limit_ns(), stream};
-  cudaError_t e = dsa::launch_sparse_mla(p);
-  if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
-  return DSA_OK;
+  // A workspace smaller than dsa_workspace_size only lowers how many CTAs share a row.
+  dsa::MlaLaunch p{q,     kv,  cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, static_cast<float*>(ws),
+                   ws ? ws_bytes : 0, dev->sm_count, wait_limit_ns(), stream};
+  return run_sparse_mla(p);
 }
 
 int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q, const dsa_bf16* kv,
@@ -309,15 +321,15 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   float* scores = reinterpret_cast<float*>(base + ws_indexer(T));
   int32_t* idx_ws = reinterpret_cast<int32_t*>(base + ws_indexer(T) + align_up(size_t(T) * size_t(ld) * 4, 256));
   int32_t* idx = idx_out ? idx_out : idx_ws;
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(idx_ws) + align_up(size_t(T) * size_t(topk) * 4, 256));
 
   if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, ld, plan, stream, dev->sm_count)))
     return rc;
   cudaError_t e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, stream);
   if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
-  dsa::MlaLaunch p{q, kv, cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, wait_limit_ns(), stream};
-  e = dsa::launch_sparse_mla(p);
-  if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
-  return DSA_OK;
+  dsa::MlaLaunch p{q,    kv,  cache_rows,        kv_start,      idx,           T,     topk, scale,
+                   o_lat, lse, part,              ws_mla(T, topk), dev->sm_count, wait_limit_ns(), stream};
+  return run_sparse_mla(p);
 }
 
 int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,

@@ -60,8 +60,8 @@ cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_
 
 // ------------------------------------------------------------------ sparse MLA
 struct MlaLaunch {
-  const uint16_t* q;
-  const uint16_t* kv;
+  const uint16_t* q;   // [T,64,576]: read through a tensor map (64-row boxes)
+  const uint16_t* kv;  // [cache_rows,576]: gathered with 16-byte cp.async
   int64_t cache_rows;
   const int64_t* kv_start;
   const int32_t* idx;
@@ -70,13 +70,17 @@ struct MlaLaunch {
   float scale;
   float* o_lat;
   float* lse;
+  float* part;        // split partials (may be null: one CTA per row)
+  size_t part_bytes;
+  int sm_count;
   unsigned long long wait_ns;
   cudaStream_t stream;
 };
-cudaError_t launch_sparse_mla(const MlaLaunch& p);
+cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q);
 
 // Shared-memory opt-in sizes, set once per device.
 cudaError_t prepare_indexer();
 cudaError_t prepare_sparse_mla();
+cudaError_t prepare_topk();
 
 }  // namespace dsa

@@ -3,22 +3,29 @@
 //   S[h,j]   = scale * (q_lat[h] . c_kv[s_j] + q_rope[h] . k_rope[s_j])
 //   o_lat[h] = sum_j softmax_j(S[h,:]) c_kv[s_j],   lse[h] = log sum_j exp S[h,j]
 //
-// ("From a trillion dot products to two thousand: how DSA breaks N^2", "DSA full flow": full Q.K, softmax and the
-// value mix over the selected 2048 only; "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2",
+// ("From a trillion dot products to two thousand: how DSA breaks N^2", "DSA
+// full flow": full Q.K, softmax and the value mix over the selected 2048
+// only; "2026 LLM architecture overview (2): DSA and MoE of GLM 5 / DSV3.2",
 // section 2.1: 64 heads, kv_lora_rank 512, rope 64, qk_head_dim 256.)
 //
-// One CTA per query row.  The selected 1152-byte rows are gathered 128 at a
-// time with 16-byte cp.async into a 128-byte-swizzled tile (9 column chunks
-// of 64).  Each tile is used twice by the tensor cores without moving it:
-//  * S^T = K . Q^T   (M = 128 keys, N = 64 heads, K = 576): A = tile, K-major;
-//    B = q (resident, 9 chunks), K-major.  S^T lands in TMEM: lane = key.
-//  * O^T += V^T . P^T (M = 128 latent dims x 4, N = 64 heads, K = 128 keys):
-//    A = the same tile read MN-major (the latent dims are contiguous), B = P
-//    written as bf16 into the tile's rope chunk, which is dead once S exists.
-// Softmax state is fp32: each thread owns one key row of S^T; the per-head
-// max and sum across the 128 keys use a 62-shuffle reduce-scatter per warp
-// plus a 4-way combine in shared memory.  The running max is updated lazily
-// (only when a tile max exceeds it by 2^8), so O in TMEM is rescaled rarely.
+// One CTA per (query row, split of its selected positions); 9 warps:
+//  * warps 0..3, producers: q (64 x 576) once by TMA, then a stream of 32 KB
+//    slots through a 4-deep ring.  A slot is two 64-column chunks of 128
+//    selected rows in the 128-byte-swizzled layout the tensor cores read,
+//    filled with 16-byte cp.async (an empty index slot is zero-filled).  Each
+//    thread keeps two slots in flight and retires a slot after its own copies
+//    land (wait_group, proxy fence, mbarrier arrive).  Per tile t the stream
+//    carries its key chunks 0..8 (five slots) and, one tile later, its latent
+//    chunks 0..7 again (four slots) for the value product: the rows cross L2
+//    twice instead of holding a 144 KB tile.
+//  * warp 4, MMA issuer: S^T_t = K_t . Q^T (M = 128 keys, N = 64 heads,
+//    K = 576) into one of two TMEM buffers, one tile ahead of
+//    O^T += V_t^T . P_t^T (M = 128 latent dims x 4, N = 64, K = 128), with V
+//    read MN-major straight from the slot.
+//  * warps 5..8, softmax: each thread owns one key row of S^T; fp32 running
+//    max and sum per head (62-shuffle reduce-scatter per warp + 4-way combine),
+//    lazy rescale of O when a tile max passes the running max by 2^8; P goes
+//    to shared memory as bf16 for the value product.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -31,26 +38,42 @@ namespace {
 
 constexpr int kRow = 576;
 constexpr int kTileKeys = 128;
-constexpr int kChunkKeyBytes = kTileKeys * 128;  // 16 KB: 128 rows x 64 columns
+constexpr int kChunkBytes = kTileKeys * 128;     // 16 KB: 128 rows x 64 columns, 128B-swizzled
+constexpr int kSlotBytes = 2 * kChunkBytes;      // two chunks
+constexpr int kNumSlots = 4;
 constexpr int kQChunkBytes = 64 * 128;           // 8 KB: 64 heads x 64 columns
-constexpr int kTileOff = 0;
-constexpr int kQOff = 9 * kChunkKeyBytes;                // 147456
-constexpr int kMiscOff = kQOff + 9 * kQChunkBytes;       // 221184
-constexpr int kRedOff = kMiscOff;                        // float red[4][64]
-constexpr int kMUseOff = kRedOff + 4 * 64 * 4;           // float m_use[64]
-constexpr int kLOff = kMUseOff + 64 * 4;                 // float l_run[64]
-constexpr int kAlphaOff = kLOff + 64 * 4;                // float alpha[64]
-constexpr int kIdxOff = kAlphaOff + 64 * 4;              // long long row[128] (absolute cache row or -1)
-constexpr int kBarOff = kIdxOff + 128 * 8;               // 5 mbarriers
-constexpr int kSlotOff = kBarOff + 5 * 8;                // tmem slot, abort flag
+constexpr int kKeySlots = 5;                     // chunks 0..8 of a key tile
+constexpr int kValSlots = 4;                     // chunks 0..7 of a value tile
+constexpr int kQOff = 0;                                    // 9 x 8 KB
+constexpr int kRingOff = 9 * kQChunkBytes;                  // 73728
+constexpr int kPOff = kRingOff + kNumSlots * kSlotBytes;    // 204800: P, 128 keys x 64 heads bf16
+constexpr int kMiscOff = kPOff + kChunkBytes;               // 221184
+constexpr int kRedOff = kMiscOff;                           // float red[4][64]
+constexpr int kMUseOff = kRedOff + 4 * 64 * 4;              // float m_use[64]
+constexpr int kLOff = kMUseOff + 64 * 4;                    // float l_run[64]
+constexpr int kAlphaOff = kLOff + 64 * 4;                   // float alpha[64]
+constexpr int kYOff = kAlphaOff + 64 * 4;                   // int y[2][128]: cache rows of two tiles
+constexpr int kBarOff = kYOff + 2 * 128 * 4;                // mbarriers
+constexpr int kNumBars = 1 + 2 * kNumSlots + 2 + 1 + 1 + 1; // q, slots full/empty, s_full x2, p_full, p_free, drain
+constexpr int kSlotOff = kBarOff + kNumBars * 8;            // tmem slot, abort flag
 constexpr int kSmemBytes = kSlotOff + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 0;    // S^T: 64 columns
-constexpr uint32_t kOCol = 64;   // O^T: 4 tiles x 64 columns
+constexpr uint32_t kSCol = 0;     // S^T buffers: columns 0..63 and 64..127
+constexpr uint32_t kOCol = 128;   // O^T: 4 tiles x 64 columns
 constexpr float kLazyRescale = 8.0f;  // log2 units
+constexpr int kPartFloats = 64 * 512 + 2 * 64;  // one split's O, running max, running sum
+constexpr int kMlaThreads = 288;
+constexpr int kSlotsInFlight = 2;  // per producer thread
 
 __device__ __forceinline__ float fmax_(float a, float b) { return a > b ? a : b; }
+
+// 2^x with the SFU instruction (ex2.approx: relative error ~2^-22; 2^-inf = +0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Reduce 64 per-thread values across the warp; lane L returns heads 2L, 2L+1.
 template <bool kMax>
@@ -135,10 +158,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& rlo, 
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-__global__ void __launch_bounds__(160, 1)
-    sparse_mla_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ kv, int64_t cache_rows,
-                      const int64_t* __restrict__ kv_start, const int32_t* __restrict__ idx, int topk,
-                      float scale_log2, float* __restrict__ o_lat, float* __restrict__ lse, WaitLimit lim) {
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    sparse_mla_kernel(const uint16_t* __restrict__ kv, const __grid_constant__ CUtensorMap tmap_q,
+                      int64_t cache_rows, const int64_t* __restrict__ kv_start, const int32_t* __restrict__ idx,
+                      int topk, float scale_log2, float* __restrict__ o_lat, float* __restrict__ lse, int splits,
+                      int tiles_per_split, float* __restrict__ part, WaitLimit lim) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -146,28 +170,45 @@ __global__ void __launch_bounds__(160, 1)
   float* m_use = reinterpret_cast<float*>(smem + kMUseOff);
   float* l_run = reinterpret_cast<float*>(smem + kLOff);
   float* alpha_s = reinterpret_cast<float*>(smem + kAlphaOff);
-  long long* row_s = reinterpret_cast<long long*>(smem + kIdxOff);
-  const uint32_t kv_full = sbase + kBarOff, s_full = kv_full + 8, p_full = kv_full + 16, kv_free = kv_full + 24;
-  const uint32_t drain = kv_full + 32;
+  const uint32_t bar0 = sbase + kBarOff;
+  const uint32_t q_full = bar0;
+  auto slot_full = [&](int j) { return bar0 + 8u * (1 + j); };
+  auto slot_empty = [&](int j) { return bar0 + 8u * (1 + kNumSlots + j); };
+  auto s_full = [&](int b) { return bar0 + 8u * (1 + 2 * kNumSlots + b); };
+  const uint32_t p_full = bar0 + 8u * (3 + 2 * kNumSlots);
+  const uint32_t p_free = bar0 + 8u * (4 + 2 * kNumSlots);
+  const uint32_t drain = bar0 + 8u * (5 + 2 * kNumSlots);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSlotOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSlotOff + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x;
-  const int ntiles = (topk + kTileKeys - 1) / kTileKeys;
+  // CTA = (query row i, split sp); the split owns tiles [t_first, t_first + ntiles).
+  const int i = blockIdx.x / splits;
+  const int sp = blockIdx.x - i * splits;
+  const int ntiles_row = (topk + kTileKeys - 1) / kTileKeys;
+  const int t_first = sp * tiles_per_split;
+  const int ntiles = max(0, min(ntiles_row, t_first + tiles_per_split) - t_first);
+  const long long ks = kv_start[i];
+  const int32_t* irow = idx + (long long)i * topk;
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 128);
-    mbar_init(s_full, 1);
+    mbar_init(q_full, 1);
+    for (int j = 0; j < kNumSlots; ++j) {
+      mbar_init(slot_full(j), 128);  // one arrival per producer thread
+      mbar_init(slot_empty(j), 1);
+    }
+    mbar_init(s_full(0), 1);
+    mbar_init(s_full(1), 1);
     mbar_init(p_full, 128);
-    mbar_init(kv_free, 1);
+    mbar_init(p_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&tmap_q);
   }
-  if (threadIdx.x < 64) {
-    m_use[threadIdx.x] = -INFINITY;
-    l_run[threadIdx.x] = 0.f;
+  if (threadIdx.x >= 160 && threadIdx.x < 224) {
+    m_use[threadIdx.x - 160] = -INFINITY;
+    l_run[threadIdx.x - 160] = 0.f;
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -178,37 +219,141 @@ __global__ void __launch_bounds__(160, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp < 4) {
+    // ---------------------------------------------------------------- producers (warps 0..3)
+    const int pt = threadIdx.x;  // 0..127
+    int* y_s = reinterpret_cast<int*>(smem + kYOff);
+    if (pt == 0 && ntiles > 0) {
+      mbar_arrive_expect_tx(q_full, 9 * kQChunkBytes);
+      for (int c = 0; c < 9; ++c) tma_load_2d(sbase + kQOff + c * kQChunkBytes, &tmap_q, q_full, 64 * c, i * 64);
+    }
+    // two-chunk slot: 16-byte segment g2 of chunk h2 for rows r2 + 8j; one-chunk slot: segment g1 of rows r1 + 16j
+    const int h2 = (pt >> 3) & 1, g2 = pt & 7, r2 = pt >> 4;
+    const int g1 = pt & 7, r1 = pt >> 3;
+    int slot = 0, n_issued = 0, n_retired = 0;
+    uint32_t sphase = 0;
+    bool ok = true;
+    auto retire = [&](int keep) {  // arrive for every issued slot but the newest `keep`
+      if (n_issued - n_retired <= keep) return;
+      if (keep >= kSlotsInFlight) cp_async_wait_group<kSlotsInFlight>();
+      else cp_async_wait_group<0>();
+      fence_proxy_async_smem();
+      while (n_issued - n_retired > keep) {
+        mbar_arrive(slot_full(n_retired % kNumSlots));
+        ++n_retired;
+      }
+    };
+    auto issue_slot = [&](int c0, int nchunks, const int* yrow) {
+      if (!mbar_wait(slot_empty(slot), sphase ^ 1u, lim, abort_flag)) return false;
+      const uint32_t sb = sbase + kRingOff + slot * kSlotBytes;
+      if (nchunks == 2) {
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+          const int row = r2 + 8 * j;
+          const int y = yrow[row];
+          const uint32_t dst = sb + h2 * kChunkBytes + row * 128 + ((g2 ^ (row & 7)) << 4);
+          cp_async_16(dst, y >= 0 ? kv + (long long)y * kRow + 64 * (c0 + h2) + 8 * g2 : kv, y >= 0);
+        }
+      } else {
+#pragma unroll 4
+        for (int j = 0; j < 8; ++j) {
+          const int row = r1 + 16 * j;
+          const int y = yrow[row];
+          const uint32_t dst = sb + row * 128 + ((g1 ^ (row & 7)) << 4);
+          cp_async_16(dst, y >= 0 ? kv + (long long)y * kRow + 64 * c0 + 8 * g1 : kv, y >= 0);
+        }
+      }
+      cp_async_commit();
+      ++n_issued;
+      if (++slot == kNumSlots) {
+        slot = 0;
+        sphase ^= 1u;
+      }
+      retire(kSlotsInFlight);
+      return true;
+    };
+    for (int s = 0; s <= ntiles && ok; ++s) {
+      if (s < ntiles) {
+        // cache rows of tile s (-1: empty or out of range) into y_s[s & 1]
+        named_bar_sync(2, 128);  // every producer is done with the tile that used this buffer
+        {
+          const int slot_i = (t_first + s) * kTileKeys + pt;
+          int yy = -1;
+          if (slot_i < topk) {
+            const int v = irow[slot_i];
+            if (v >= 0) {
+              if (ks + v < cache_rows) yy = int(ks + v);
+              else raise_status(kStatusBadRow);
+            }
+          }
+          y_s[(s & 1) * 128 + pt] = yy;
+        }
+        named_bar_sync(2, 128);
+        for (int p = 0; p < kKeySlots && ok; ++p) ok = issue_slot(2 * p, p < 4 ? 2 : 1, y_s + (s & 1) * 128);
+      }
+      if (s >= 1) {
+        for (int p = 0; p < kValSlots && ok; ++p) ok = issue_slot(2 * p, 2, y_s + ((s - 1) & 1) * 128);
+      }
+    }
+    retire(0);  // all copies landed and every issued slot arrived
+  } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && ntiles > 0) {
       const uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_o = idesc_bf16(128, 64, 1, 1);
-      const uint32_t tile = sbase + kTileOff, qs = sbase + kQOff, pbuf = tile + 8 * kChunkKeyBytes;
-      for (int t = 0; t < ntiles; ++t) {
-        if (!mbar_wait(kv_full, uint32_t(t & 1), lim, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 9; ++c)
+      int slot = 0;
+      uint32_t sphase = 0;
+      bool ok = mbar_wait(q_full, 0, lim, abort_flag);
+      for (int s = 0; s <= ntiles && ok; ++s) {
+        if (s < ntiles) {
+          const uint32_t d = tmem + kSCol + 64 * (s & 1);
+          for (int p = 0; p < kKeySlots && ok; ++p) {
+            if (!(ok = mbar_wait(slot_full(slot), sphase, lim, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t a0 = sbase + kRingOff + slot * kSlotBytes;
+            const int nch = p < 4 ? 2 : 1;
+            for (int h = 0; h < nch; ++h) {
+              const int c = 2 * p + h;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = smem_desc(tile + c * kChunkKeyBytes + k * 32, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(qs + c * kQChunkBytes + k * 32, 16, 1024, kSwizzle128B);
-            mma_bf16_ss(tmem + kSCol, ad, bd, idesc_s, (c | k) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = smem_desc(a0 + h * kChunkBytes + 32 * k, 16, 1024, kSwizzle128B);
+                const uint64_t bd = smem_desc(sbase + kQOff + c * kQChunkBytes + 32 * k, 16, 1024, kSwizzle128B);
+                mma_bf16_ss(d, ad, bd, idesc_s, (c | k) ? 1u : 0u);
+              }
+            }
+            mma_commit(slot_empty(slot));
+            if (++slot == kNumSlots) {
+              slot = 0;
+              sphase ^= 1u;
+            }
           }
-        mma_commit(s_full);
-        if (!mbar_wait(p_full, uint32_t(t & 1), lim, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int m = 0; m < 4; ++m)
+          if (!ok) break;
+          mma_commit(s_full(s & 1));
+        }
+        if (s >= 1) {
+          const int t = s - 1;
+          if (!(ok = mbar_wait(p_full, uint32_t(t & 1), lim, abort_flag))) break;
+          tc_fence_after();
+          for (int m = 0; m < kValSlots && ok; ++m) {
+            if (!(ok = mbar_wait(slot_full(slot), sphase, lim, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t a0 = sbase + kRingOff + slot * kSlotBytes;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            // V^T tile m: latent dims 128m..128m+127 are chunks 2m, 2m+1 (LBO apart); keys 16k..16k+15.
-            const uint64_t ad = smem_desc(tile + (2 * m) * kChunkKeyBytes + k * 2048, kChunkKeyBytes, 1024,
-                                          kSwizzle128B);
-            const uint64_t bd = smem_desc(pbuf + k * 2048, kChunkKeyBytes, 1024, kSwizzle128B);
-            mma_bf16_ss(tmem + kOCol + 64 * m, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 8; ++k) {
+              // V^T: latent dims 128m..128m+127 = the slot's two chunks (LBO apart); keys 16k..16k+15
+              const uint64_t ad = smem_desc(a0 + k * 2048, kChunkBytes, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(sbase + kPOff + k * 2048, kChunkBytes, 1024, kSwizzle128B);
+              mma_bf16_ss(tmem + kOCol + 64 * m, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(slot_empty(slot));
+            if (++slot == kNumSlots) {
+              slot = 0;
+              sphase ^= 1u;
+            }
           }
-        mma_commit(kv_free);
+          if (!ok) break;
+          mma_commit(p_free);
+        }
       }
       // every MMA issued above must be complete before TMEM is released
       mma_commit(drain);
@@ -216,69 +361,33 @@ __global__ void __launch_bounds__(160, 1)
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- gather + softmax (warps 0..3)
-    const int st = threadIdx.x;  // 0..127
-    const int quarter = warp;    // TMEM lane quarter
+    // ---------------------------------------------------------------- softmax (warps 5..8)
+    const int st = threadIdx.x - 160;  // 0..127
+    const int quarter = warp & 3;     // TMEM lane quarter
     const int r = quarter * 32 + lane;
-    const long long ks = kv_start[i];
-    const int32_t* irow = idx + (long long)i * topk;
+    const int rw = st >> 5;           // slot of this warp in red[]
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
-      if (t > 0 && !mbar_wait(kv_free, uint32_t((t - 1) & 1), lim, abort_flag)) {
-        ok = false;
-        break;
+      const int slot_i = (t_first + t) * kTileKeys + r;
+      bool valid = false;
+      if (slot_i < topk) {
+        const int s = irow[slot_i];
+        valid = s >= 0 && ks + s < cache_rows;
       }
-      // stage this tile's cache rows
-      {
-        const int slot = t * kTileKeys + st;
-        long long rr = -1;
-        if (slot < topk) {
-          const int s = irow[slot];
-          if (s >= 0) {
-            if (ks + s < cache_rows) rr = ks + s;
-            else raise_status(kStatusBadRow);
-          }
-        }
-        row_s[st] = rr;
-      }
-      named_bar_sync(1, 128);
-      if (t == 0) {
-        const uint16_t* qrow = q + (long long)i * 64 * kRow;
-        for (int e = st; e < 64 * 72; e += 128) {
-          const int h = e / 72, rem = e - h * 72, c = rem >> 3, g = rem & 7;
-          const uint32_t dst = sbase + kQOff + c * kQChunkBytes + h * 128 + ((g ^ (h & 7)) << 4);
-          cp_async_16(dst, qrow + h * kRow + c * 64 + g * 8, true);
-        }
-      }
-      for (int e = st; e < kTileKeys * 72; e += 128) {
-        const int row = e / 72, rem = e - row * 72, c = rem >> 3, g = rem & 7;
-        const long long rr = row_s[row];
-        const uint32_t dst = sbase + kTileOff + c * kChunkKeyBytes + row * 128 + ((g ^ (row & 7)) << 4);
-        const uint16_t* src = rr >= 0 ? kv + rr * kRow + c * 64 + g * 8 : kv;
-        cp_async_16(dst, src, rr >= 0);
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(kv_full);
-
-      if (!mbar_wait(s_full, uint32_t(t & 1), lim, abort_flag)) {
-        ok = false;
-        break;
-      }
+      if (!(ok = mbar_wait(s_full(t & 1), uint32_t((t >> 1) & 1), lim, abort_flag))) break;
       tc_fence_after();
       float x[64];
-      const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-      tmem_ld32_sync(lane_addr + kSCol, x);
-      tmem_ld32_sync(lane_addr + kSCol + 32, x + 32);
-      const bool valid = row_s[r] >= 0;
+      tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1), x);
+      tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1) + 32, x + 32);
 #pragma unroll
       for (int h = 0; h < 64; ++h) x[h] = valid ? x[h] * scale_log2 : -INFINITY;
 
       // per-head max over the tile's 128 keys
       float r0, r1;
       reduce_scatter64<true>(x, r0, r1);
-      red[quarter * 64 + 2 * lane] = r0;
-      red[quarter * 64 + 2 * lane + 1] = r1;
+      red[rw * 64 + 2 * lane] = r0;
+      red[rw * 64 + 2 * lane + 1] = r1;
       named_bar_sync(1, 128);
       int resc = 0;
       if (st < 64) {
@@ -286,7 +395,7 @@ __global__ void __launch_bounds__(160, 1)
         const float mu = m_use[st];
         float al = 1.f;
         if (mt > -INFINITY && (mu == -INFINITY || mt > mu + kLazyRescale)) {
-          al = exp2f(mu - mt);  // 0 when mu = -inf
+          al = fast_exp2(mu - mt);  // 0 when mu = -inf
           m_use[st] = mt;
           l_run[st] *= al;
           resc = (t > 0) && (al != 1.f);
@@ -295,28 +404,11 @@ __global__ void __launch_bounds__(160, 1)
       }
       resc = bar_red_or_128(resc);  // also the barrier that publishes m_use / alpha
 
-      // probabilities (bf16 for the MMA) and their per-head sums
-      float p[64];
-      uint8_t* prow = smem + kTileOff + 8 * kChunkKeyBytes + r * 128;
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int h = g * 8 + 2 * u;
-          const float m0 = m_use[h], m1 = m_use[h + 1];
-          const float e0 = (valid && m0 > -INFINITY) ? exp2f(x[h] - m0) : 0.f;
-          const float e1 = (valid && m1 > -INFINITY) ? exp2f(x[h + 1] - m1) : 0.f;
-          w4[u] = pack_bf16x2(e0, e1, p[h], p[h + 1]);
-        }
-        *reinterpret_cast<uint4*>(prow + ((g ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      reduce_scatter64<false>(p, r0, r1);
-      red[quarter * 64 + 2 * lane] = r0;
-      red[quarter * 64 + 2 * lane + 1] = r1;
-
+      // the single P buffer and O are free once the previous value product is done
+      if (t > 0 && !(ok = mbar_wait(p_free, uint32_t((t - 1) & 1), lim, abort_flag))) break;
       if (resc) {
-        // O^T (lane = latent dim, column = head) *= alpha[head]; PV(t-1) is complete.
+        tc_fence_after();
+        // O^T (lane = latent dim, column = head) *= alpha[head]
 #pragma unroll 1
         for (int m = 0; m < 4; ++m)
 #pragma unroll 1
@@ -331,25 +423,48 @@ __global__ void __launch_bounds__(160, 1)
           }
         tmem_wait_st();
       }
+      // probabilities (bf16 for the MMA) and their per-head sums
+      float p[64];
+      uint8_t* prow = smem + kPOff + r * 128;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int h = g * 8 + 2 * u;
+          const float m0 = m_use[h], m1 = m_use[h + 1];
+          const float e0 = (valid && m0 > -INFINITY) ? fast_exp2(x[h] - m0) : 0.f;
+          const float e1 = (valid && m1 > -INFINITY) ? fast_exp2(x[h + 1] - m1) : 0.f;
+          w4[u] = pack_bf16x2(e0, e1, p[h], p[h + 1]);
+        }
+        *reinterpret_cast<uint4*>(prow + ((g ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      reduce_scatter64<false>(p, r0, r1);
+      red[rw * 64 + 2 * lane] = r0;
+      red[rw * 64 + 2 * lane + 1] = r1;
       named_bar_sync(1, 128);
       if (st < 64) l_run[st] += red[st] + red[64 + st] + red[128 + st] + red[192 + st];
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // final PV must be complete before reading O
-    if (ok && ntiles > 0) ok = mbar_wait(kv_free, uint32_t((ntiles - 1) & 1), lim, abort_flag);
+    // the last value product must be complete before O is read
+    if (ok && ntiles > 0) mbar_wait(p_free, uint32_t((ntiles - 1) & 1), lim, abort_flag);
   }
-  // All 160 threads (the MMA warp after its drain): publishes l_run / m_use and
-  // makes the abort decision uniform before the epilogue.
+  // All threads: publishes l_run / m_use and makes the abort decision uniform.
   __syncthreads();
-  if (warp < 4 && !*abort_flag) {
-    const int st = threadIdx.x;
-    const int quarter = warp;
-    {
-      tc_fence_after();
-      const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-      float* orow = o_lat + (long long)i * 64 * 512;
+  if (warp >= 5 && !*abort_flag) {
+    const int st = threadIdx.x - 160;
+    const int quarter = warp & 3;
+    tc_fence_after();
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    // one split: the normalised output; several: this split's unnormalised O with
+    // its running max (log2 units) and sum, merged by sparse_mla_combine_kernel
+    const bool direct = (splits == 1);
+    float* orow = direct ? o_lat + (long long)i * 64 * 512 : part + (long long)blockIdx.x * kPartFloats;
+    if (ntiles == 0) {
+      for (int e = st; e < 64 * 512; e += 128) orow[e] = 0.f;  // a split without tiles contributes nothing
+    } else {
 #pragma unroll 1
       for (int m = 0; m < 4; ++m) {
         const int d = 128 * m + quarter * 32 + lane;
@@ -360,14 +475,25 @@ __global__ void __launch_bounds__(160, 1)
 #pragma unroll
           for (int hh = 0; hh < 32; ++hh) {
             const int h = 32 * half + hh;
-            const float l = l_run[h];
-            orow[h * 512 + d] = l > 0.f ? o[hh] / l : 0.f;
+            if (direct) {
+              const float l = l_run[h];
+              orow[h * 512 + d] = l > 0.f ? o[hh] / l : 0.f;
+            } else {
+              orow[h * 512 + d] = o[hh];
+            }
           }
         }
       }
-      if (lse && st < 64) {
-        const float l = l_run[st];
-        lse[(long long)i * 64 + st] = l > 0.f ? (m_use[st] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+    if (st < 64) {
+      if (direct) {
+        if (lse) {
+          const float l = l_run[st];
+          lse[(long long)i * 64 + st] = l > 0.f ? (m_use[st] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+      } else {
+        orow[64 * 512 + st] = m_use[st];
+        orow[64 * 512 + 64 + st] = l_run[st];
       }
     }
   }
@@ -380,18 +506,72 @@ __global__ void __launch_bounds__(160, 1)
   }
 }
 
+// Merge the splits of each query row: with M = max_s m_s,
+//   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 of the denominator) * ln 2.
+__global__ void __launch_bounds__(512) sparse_mla_combine_kernel(const float* __restrict__ part, int splits,
+                                                                 float* __restrict__ o_lat,
+                                                                 float* __restrict__ lse) {
+  __shared__ float wgt[16][64];
+  __shared__ float inv_den[64];
+  const int i = blockIdx.x;
+  const float* p = part + (long long)i * splits * kPartFloats;
+  if (threadIdx.x < 64) {
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmax_(M, p[(long long)s * kPartFloats + 64 * 512 + h]);
+    float den = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float ms = p[(long long)s * kPartFloats + 64 * 512 + h];
+      const float w = (M == -INFINITY) ? 0.f : fast_exp2(ms - M);
+      wgt[s][h] = w;
+      den += w * p[(long long)s * kPartFloats + 64 * 512 + 64 + h];
+    }
+    inv_den[h] = den > 0.f ? 1.f / den : 0.f;
+    if (lse) lse[(long long)i * 64 + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
+  float* orow = o_lat + (long long)i * 64 * 512;
+  for (int e = threadIdx.x; e < 64 * 512; e += blockDim.x) {
+    const int h = e >> 9;
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) acc += wgt[s][h] * p[(long long)s * kPartFloats + e];
+    orow[e] = acc * inv_den[h];
+  }
+}
+
 }  // namespace
+
+// Splits per query row: enough CTAs to cover the SMs, at most one per 128-key
+// tile and at most kMaxSplits; `ws_bytes` bounds them too.
+constexpr int kMaxSplits = 16;
+inline size_t sparse_mla_part_bytes(int T, int splits) { return size_t(T) * splits * kPartFloats * 4; }
+inline int sparse_mla_ws_splits(int T, int topk) {
+  const int ntiles = (topk + kTileKeys - 1) / kTileKeys;
+  int s = T > 0 ? 320 / T : 1;
+  return s < 1 ? 1 : (s > kMaxSplits ? kMaxSplits : (s > ntiles ? ntiles : s));
+}
 
 cudaError_t prepare_sparse_mla() {
   static_assert(kSmemAlloc <= 232448, "sparse MLA shared memory exceeds the per-CTA limit");
   return cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
 }
 
-cudaError_t launch_sparse_mla(const MlaLaunch& p) {
+cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q) {
   if (p.T <= 0) return cudaSuccess;
   const float scale_log2 = p.scale * 1.4426950408889634f;
-  sparse_mla_kernel<<<p.T, 160, kSmemAlloc, p.stream>>>(p.q, p.kv, p.cache_rows, p.kv_start, p.idx, p.topk,
-                                                        scale_log2, p.o_lat, p.lse, WaitLimit{p.wait_ns});
+  const int ntiles = (p.topk + kTileKeys - 1) / kTileKeys;
+  int splits = p.sm_count > 0 ? p.sm_count / p.T : 1;
+  splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : (splits > ntiles ? ntiles : splits));
+  while (splits > 1 && (p.part == nullptr || sparse_mla_part_bytes(p.T, splits) > p.part_bytes)) --splits;
+  const int per = (ntiles + splits - 1) / splits;
+  splits = (ntiles + per - 1) / per;  // no split without tiles
+  if (int64_t(p.T) * splits > INT32_MAX) return cudaErrorInvalidValue;
+  sparse_mla_kernel<<<p.T * splits, kMlaThreads, kSmemAlloc, p.stream>>>(
+      p.kv, tmap_q, p.cache_rows, p.kv_start, p.idx, p.topk, scale_log2, p.o_lat, p.lse, splits, per, p.part,
+      WaitLimit{p.wait_ns});
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  sparse_mla_combine_kernel<<<p.T, 512, 0, p.stream>>>(p.part, splits, p.o_lat, p.lse);
   return cudaGetLastError();
 }
 

@@ -43,13 +43,15 @@ def gpu_topk(scores_np_f32, n_vis, k):
     return idx.cpu().numpy()
 
 
-def gpu_attention(d, idx_np, scale=SCALE):
+def gpu_attention(d, idx_np, scale=SCALE, split=False):
+    """split=True passes the workspace, so rows may be spread over several CTAs."""
     import torch
     T, k = idx_np.shape
     idx = torch.from_numpy(np.ascontiguousarray(idx_np, np.int32)).cuda()
     o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
     lse = torch.full((T, 64), float("nan"), dtype=torch.float32, device="cuda")
-    B.dsa_sparse_mla_attn(d["q"], d["kv"], d["kv_start"], idx, scale, o, lse)
+    ws = B.workspace(B.DSA_OP_SPARSE_MLA, T, 0, k) if split else None
+    B.dsa_sparse_mla_attn(d["q"], d["kv"], d["kv_start"], idx, scale, o, lse, ws)
     B.dsa_sync_status()
     return o.cpu().numpy(), lse.cpu().numpy()
 

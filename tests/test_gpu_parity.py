@@ -117,11 +117,47 @@ def test_topk_bit_exact(kind, k):
         assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
 
 
-def test_topk_long_row_exact():
-    n, k = 131072, 2048
-    S = _topk_case("normal", n, 5)[None]
-    ref = oracle.topk(S.astype(np.float64), np.array([n], np.int32), k)
-    assert np.array_equal(gpu_topk(S, [n], k), ref)
+@pytest.mark.parametrize("path", ["filtered", "full"])
+def test_topk_long_rows_exact(path, monkeypatch):
+    if path == "full":
+        monkeypatch.setenv("DSA_TOPK_KERNEL", "row")
+    lens = [131072, 204800, 65537]
+    ld = 204800
+    S = np.full((3, ld), np.nan, np.float32)
+    for i, n in enumerate(lens):
+        S[i, :n] = _topk_case("normal" if i != 2 else "ties", n, 5 + i)
+    n_vis = np.array(lens, np.int32)
+    ref = oracle.topk(S.astype(np.float64), n_vis, 2048)
+    assert np.array_equal(gpu_topk(S, n_vis, 2048), ref)
+
+
+def test_topk_filter_fallbacks():
+    # rows where the sample threshold admits too many keys (all equal, sorted
+    # ascending with a constant tail) or where the sample misses the top keys
+    n, k = 50000, 2048
+    S = np.zeros((4, n), np.float32)
+    S[0] = 1.0                                           # every key equal
+    S[1] = np.arange(n, dtype=np.float32)                # increasing: top keys at the end
+    S[2, :] = 0.5
+    S[2, 7::12] = 2.0                                    # a regular comb between sample points
+    r = np.random.default_rng(3)
+    S[3] = r.standard_normal(n).astype(np.float32)
+    S[3, r.choice(n, 3000, replace=False)] = 9.0         # 3000 ties above everything else
+    n_vis = np.full(4, n, np.int32)
+    ref = oracle.topk(S.astype(np.float64), n_vis, k)
+    assert np.array_equal(gpu_topk(S, n_vis, k), ref)
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "wide"])
+def test_topk_full_radix_path_bit_exact(kind, monkeypatch):
+    monkeypatch.setenv("DSA_TOPK_KERNEL", "row")
+    lens = [1, 2047, 2048, 2049, 5000, 20000]
+    S = np.full((len(lens), 20000), np.nan, np.float32)
+    for i, n in enumerate(lens):
+        S[i, :n] = _topk_case(kind, n, seed=100 + i)
+    n_vis = np.array(lens, np.int32)
+    ref = oracle.topk(S.astype(np.float64), n_vis, 2048)
+    assert np.array_equal(gpu_topk(S, n_vis, 2048), ref)
 
 
 # ---------------------------------------------------------------------------- attention
@@ -136,14 +172,31 @@ def _attention_case(seed, L=3000, T=5, k=2048, pad=(0, 100, 1900, 2047, 0)):
     return c, idx
 
 
-def test_attention_matches_oracle_on_given_indices():
+@pytest.mark.parametrize("split", [False, True])
+def test_attention_matches_oracle_on_given_indices(split):
     c, idx = _attention_case(41)
     o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
-    o, lse = gpu_attention(to_dev(c), idx)
+    o, lse = gpu_attention(to_dev(c), idx, split=split)
     assert_attention_close(o, lse, o_ref, lse_ref)
 
 
-def test_attention_ragged_topk_and_gaps():
+def test_attention_split_with_empty_tiles_and_large_logits():
+    # splits whose tiles hold no valid index, and logits large enough that the
+    # splits' running maxima differ by far more than the lazy-rescale margin
+    c = wl.make_case_numpy([3000], [(0, 3000)] * 3, seed=46, n_plant=0)
+    c.q = wl.bf16_from_f32(wl.bf16_to_f32(c.q) * 6.0)
+    r = np.random.default_rng(46)
+    idx = np.full((3, 2048), -1, np.int32)
+    idx[0, :130] = np.sort(r.choice(3000, 130, replace=False))          # only the first tiles
+    idx[1, 1900:] = np.sort(r.choice(3000, 148, replace=False))         # only the last tile
+    idx[2] = np.sort(r.choice(3000, 2048, replace=False))
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx, split=True)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_attention_ragged_topk_and_gaps(split):
     # topk not a multiple of 128, -1 holes inside the list, unsorted entries
     c = wl.make_case_numpy([800], [(0, 800)] * 3, seed=43, n_plant=0)
     r = np.random.default_rng(43)
@@ -154,18 +207,19 @@ def test_attention_ragged_topk_and_gaps():
     idx[1, 5] = 123                     # single key: o = c_kv[123]
     idx[2, 150:] = -1
     o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
-    o, lse = gpu_attention(to_dev(c), idx)
+    o, lse = gpu_attention(to_dev(c), idx, split=split)
     assert_attention_close(o, lse, o_ref, lse_ref)
 
 
-def test_attention_empty_row_and_large_logits():
+@pytest.mark.parametrize("split", [False, True])
+def test_attention_empty_row_and_large_logits(split):
     c = wl.make_case_numpy([500], [(0, 500)] * 2, seed=44, n_plant=0)
     qf = wl.bf16_to_f32(c.q) * 8.0     # logits up to ~ +-40: exercises the lazy rescale
     c.q = wl.bf16_from_f32(qf)
     idx = np.full((2, 512), -1, np.int32)
     idx[0] = np.arange(500, dtype=np.int32).tolist() + [-1] * 12
     o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
-    o, lse = gpu_attention(to_dev(c), idx)
+    o, lse = gpu_attention(to_dev(c), idx, split=split)
     assert_attention_close(o, lse, o_ref, lse_ref)
     assert (o[1] == 0).all() and np.isneginf(lse[1]).all()
 
