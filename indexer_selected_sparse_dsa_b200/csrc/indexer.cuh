@@ -15,8 +15,9 @@
 // columns per query from TMEM and reduces them with w into one fp32 score,
 // so the head reduction needs no cross-thread traffic.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
-// and MMA issuer, warps 2..5 = epilogue.  Persistent grid.
+// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
+// and MMA issuer, warps 2..9 = epilogue (two warps per TMEM lane quarter, each
+// taking every other query of the tile).  Persistent grid.
 #pragma once
 #include <cuda.h>
 
@@ -180,6 +181,9 @@ struct UnitIter {
 };
 
 // ------------------------------------------------------------------ main kernel
+constexpr int kEpiWarps = 8;
+constexpr int kIdxThreads = 64 + 32 * kEpiWarps;
+
 template <int QMAX, int STAGES, int QBUF>
 struct IdxSmem {
   static constexpr int kQBufBytes = QMAX * 2 * kQBoxBytes;  // two halves
@@ -197,7 +201,7 @@ struct IdxSmem {
 };
 
 template <int QMAX, int STAGES, int QBUF>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const uint16_t* __restrict__ w, const int32_t* __restrict__ n_vis,
                    const PlanHeader* __restrict__ hdr, const PlanTile* __restrict__ tiles, float* __restrict__ scores,
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(afull_bar(b), 1);
-      mbar_init(aempty_bar(b), 4);  // one arrival per epilogue warp
+      mbar_init(aempty_bar(b), kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -343,10 +347,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain_bar, 0, lim, nullptr);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..5)
-    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    // ---------------------------------------------------------------- epilogue (warps 2..9)
+    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;     // queries half, half + 2, half + 4, ...
     const int row = quarter * 32 + lane;
-    const int et = threadIdx.x - 64;  // 0..127
+    const int et = threadIdx.x - 64;      // 0 .. 32 * kEpiWarps - 1
     UnitIter it;
     it.sweep = sweep;
     int prev_tile = -1, ab = 0;
@@ -355,25 +360,49 @@ __global__ void __launch_bounds__(192, 1)
     while (ok) {
       const int nq = it.cur.nq;
       if (it.tile != prev_tile) {
-        named_bar_sync(1, 128);
-        for (int e = et; e < nq * 32; e += 128)
+        named_bar_sync(1, 32 * kEpiWarps);
+        for (int e = et; e < nq * 32; e += 32 * kEpiWarps)
           w_s[e] = bf16_bits_to_float(w[(long long)it.cur.q0 * 32 + e]);
         if (et < nq) nv_s[et] = n_vis[it.cur.q0 + et];
-        named_bar_sync(1, 128);
+        named_bar_sync(1, 32 * kEpiWarps);
         prev_tile = it.tile;
       }
       if (!mbar_wait(afull_bar(ab), aphase, lim, abort_flag)) break;
       tc_fence_after();
       const long long s = (long long)it.kt * kKeysPerUnit + row;
       const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
-      for (int qi = 0; qi < nq; ++qi) {
-        float v[32];
-        tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
-        const float* wq = w_s + qi * 32;
-        float acc = 0.f;
+      // this warp's queries, two per TMEM wait: qi = half, half + 2 (then + 4, + 6)
+      for (int qi = half; qi < nq; qi += 4) {
+        const int qj = qi + 2;
+        float v[64];
+        if (qj < nq) {
+          tmem_ld32x2_sync(tbase + uint32_t(qi * 32), tbase + uint32_t(qj * 32), v);
+        } else {
+          tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
+        }
+        const float4* w0 = reinterpret_cast<const float4*>(w_s + qi * 32);
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) acc = fmaf(wq[h], v[h], acc);
-        if (s < nv_s[qi]) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = acc;
+        for (int h4 = 0; h4 < 8; ++h4) {
+          const float4 c = w0[h4];
+          a0 = fmaf(c.x, v[4 * h4], a0);
+          a0 = fmaf(c.y, v[4 * h4 + 1], a0);
+          a0 = fmaf(c.z, v[4 * h4 + 2], a0);
+          a0 = fmaf(c.w, v[4 * h4 + 3], a0);
+        }
+        if (s < nv_s[qi]) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = a0;
+        if (qj < nq) {
+          const float4* w1 = reinterpret_cast<const float4*>(w_s + qj * 32);
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 c = w1[h4];
+            a1 = fmaf(c.x, v[32 + 4 * h4], a1);
+            a1 = fmaf(c.y, v[32 + 4 * h4 + 1], a1);
+            a1 = fmaf(c.z, v[32 + 4 * h4 + 2], a1);
+            a1 = fmaf(c.w, v[32 + 4 * h4 + 3], a1);
+          }
+          if (s < nv_s[qj]) scores[(long long)(it.cur.q0 + qj) * score_ld + s] = a1;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -408,7 +437,7 @@ cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUt
   using L = IdxSmem<QMAX, STAGES, QBUF>;
   auto* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<const PlanTile*>(reinterpret_cast<const uint8_t*>(p.plan) + sizeof(PlanHeader));
-  indexer_kernel<QMAX, STAGES, QBUF><<<p.grid, 192, L::kAlloc, p.stream>>>(
+  indexer_kernel<QMAX, STAGES, QBUF><<<p.grid, kIdxThreads, L::kAlloc, p.stream>>>(
       tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, WaitLimit{p.wait_ns});
   return cudaGetLastError();
 }

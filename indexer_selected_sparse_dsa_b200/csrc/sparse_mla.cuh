@@ -12,9 +12,10 @@
 //  * warps 0..3, producers: q (64 x 576) once by TMA, then a stream of 32 KB
 //    slots through a 4-deep ring.  A slot is two 64-column chunks of 128
 //    selected rows in the 128-byte-swizzled layout the tensor cores read,
-//    filled with 16-byte cp.async (an empty index slot is zero-filled).  Each
-//    thread keeps two slots in flight and retires a slot after its own copies
-//    land (wait_group, proxy fence, mbarrier arrive).  Per tile t the stream
+//    filled with 16-byte cp.async (an empty index slot is zero-filled); each
+//    thread's copies arrive on the slot's mbarrier when they land, so every
+//    free slot of the ring is in flight; the rows of tile t+1 are prefetched
+//    into L2 while tile t is staged.  Per tile t the stream
 //    carries its key chunks 0..8 (five slots) and, one tile later, its latent
 //    chunks 0..7 again (four slots) for the value product: the rows cross L2
 //    twice instead of holding a 144 KB tile.
@@ -64,7 +65,6 @@ constexpr uint32_t kOCol = 128;   // O^T: 4 tiles x 64 columns
 constexpr float kLazyRescale = 8.0f;  // log2 units
 constexpr int kPartFloats = 64 * 512 + 2 * 64;  // one split's O, running max, running sum
 constexpr int kMlaThreads = 288;
-constexpr int kSlotsInFlight = 2;  // per producer thread
 
 __device__ __forceinline__ float fmax_(float a, float b) { return a > b ? a : b; }
 
@@ -227,55 +227,37 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_arrive_expect_tx(q_full, 9 * kQChunkBytes);
       for (int c = 0; c < 9; ++c) tma_load_2d(sbase + kQOff + c * kQChunkBytes, &tmap_q, q_full, 64 * c, i * 64);
     }
-    // two-chunk slot: 16-byte segment g2 of chunk h2 for rows r2 + 8j; one-chunk slot: segment g1 of rows r1 + 16j
-    const int h2 = (pt >> 3) & 1, g2 = pt & 7, r2 = pt >> 4;
-    const int g1 = pt & 7, r1 = pt >> 3;
-    int slot = 0, n_issued = 0, n_retired = 0;
+    // Thread pt copies 16-byte segment g of chunk half h for rows r + 8j (j < 16), in
+    // every slot: the swizzled destination offset is the same for all its rows.
+    const int h = (pt >> 3) & 1, g = pt & 7, r = pt >> 4;
+    const uint32_t thr_off = uint32_t(h * kChunkBytes + r * 128 + ((g ^ (r & 7)) << 4));
+    const char* kvb = reinterpret_cast<const char*>(kv);
+    const char* cur[16];
+    const char* prev[16];
+    uint32_t cur_skip = 0u, prev_skip = 0u;  // bit j: row r + 8j is empty (zero-filled)
+    int slot = 0;
     uint32_t sphase = 0;
     bool ok = true;
-    auto retire = [&](int keep) {  // arrive for every issued slot but the newest `keep`
-      if (n_issued - n_retired <= keep) return;
-      if (keep >= kSlotsInFlight) cp_async_wait_group<kSlotsInFlight>();
-      else cp_async_wait_group<0>();
-      fence_proxy_async_smem();
-      while (n_issued - n_retired > keep) {
-        mbar_arrive(slot_full(n_retired % kNumSlots));
-        ++n_retired;
-      }
-    };
-    auto issue_slot = [&](int c0, int nchunks, const int* yrow) {
+    // copy chunk `chunk` (plus h) of the rows in `rows` into the next slot
+    auto issue_slot = [&](int chunk, bool active, const char* const* rows, uint32_t skip) {
       if (!mbar_wait(slot_empty(slot), sphase ^ 1u, lim, abort_flag)) return false;
-      const uint32_t sb = sbase + kRingOff + slot * kSlotBytes;
-      if (nchunks == 2) {
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j) {
-          const int row = r2 + 8 * j;
-          const int y = yrow[row];
-          const uint32_t dst = sb + h2 * kChunkBytes + row * 128 + ((g2 ^ (row & 7)) << 4);
-          cp_async_16(dst, y >= 0 ? kv + (long long)y * kRow + 64 * (c0 + h2) + 8 * g2 : kv, y >= 0);
-        }
-      } else {
-#pragma unroll 4
-        for (int j = 0; j < 8; ++j) {
-          const int row = r1 + 16 * j;
-          const int y = yrow[row];
-          const uint32_t dst = sb + row * 128 + ((g1 ^ (row & 7)) << 4);
-          cp_async_16(dst, y >= 0 ? kv + (long long)y * kRow + 64 * c0 + 8 * g1 : kv, y >= 0);
-        }
+      if (active) {
+        const uint32_t dst = sbase + kRingOff + slot * kSlotBytes + thr_off;
+        const int col = (chunk + h) * 128 + g * 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cp_async_16_or_zero(dst + j * 1024, rows[j] + col, (skip >> j) & 1u);
       }
-      cp_async_commit();
-      ++n_issued;
+      cp_async_arrive_noinc(slot_full(slot));  // arrives when this thread's copies have landed
       if (++slot == kNumSlots) {
         slot = 0;
         sphase ^= 1u;
       }
-      retire(kSlotsInFlight);
       return true;
     };
     for (int s = 0; s <= ntiles && ok; ++s) {
       if (s < ntiles) {
         // cache rows of tile s (-1: empty or out of range) into y_s[s & 1]
-        named_bar_sync(2, 128);  // every producer is done with the tile that used this buffer
+        named_bar_sync(2, 128);  // every producer is done reading this buffer's previous tile
         {
           const int slot_i = (t_first + s) * kTileKeys + pt;
           int yy = -1;
@@ -287,15 +269,35 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             }
           }
           y_s[(s & 1) * 128 + pt] = yy;
+          // pull the next tile's rows into L2 now, so its slot loads are L2 hits
+          const int slot_n = slot_i + kTileKeys;
+          if (s + 1 < ntiles && slot_n < topk) {
+            const int v = irow[slot_n];
+            if (v >= 0 && ks + v < cache_rows) prefetch_l2_bulk(kv + (ks + v) * kRow, kRow * 2);
+          }
         }
         named_bar_sync(2, 128);
-        for (int p = 0; p < kKeySlots && ok; ++p) ok = issue_slot(2 * p, p < 4 ? 2 : 1, y_s + (s & 1) * 128);
+        cur_skip = 0u;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int y = y_s[(s & 1) * 128 + r + 8 * j];
+          cur[j] = kvb + (long long)(y >= 0 ? y : 0) * (kRow * 2);
+          cur_skip |= (y < 0 ? 1u : 0u) << j;
+        }
+#pragma unroll
+        for (int p = 0; p < kKeySlots; ++p)
+          if (ok) ok = issue_slot(2 * p, p < 4 || h == 0, cur, cur_skip);  // the rope slot has one chunk
       }
       if (s >= 1) {
-        for (int p = 0; p < kValSlots && ok; ++p) ok = issue_slot(2 * p, 2, y_s + ((s - 1) & 1) * 128);
+#pragma unroll
+        for (int p = 0; p < kValSlots; ++p)
+          if (ok) ok = issue_slot(2 * p, true, prev, prev_skip);
       }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) prev[j] = cur[j];
+      prev_skip = cur_skip;
     }
-    retire(0);  // all copies landed and every issued slot arrived
+    cp_async_wait_all();  // no copy may still be in flight when the CTA exits
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && ntiles > 0) {
