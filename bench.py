@@ -196,6 +196,24 @@ def whole_job_rate(rows_per_rank: int, world: int, ms_per_step: float) -> float:
     return rows_per_rank * world / (ms_per_step * 1e-3)
 
 
+def forward_streams(T: int, max_n: int) -> bool:
+    """dsa_forward's rule: stream scores into the selector when the score matrix
+    would exceed 8 GB."""
+    mode = os.environ.get("DSA_FORWARD_MODE")
+    if mode in ("stream", "materialize"):
+        return mode == "stream"
+    return T * ((max_n + 3) // 4 * 4) * 4 > (8 << 30)
+
+
+def launches_per_step(T: int, k: int, streams: bool, sms: int) -> int:
+    """Kernels of this library one dsa_forward launches: indexer plan, indexer,
+    top-k (materialised path), attention, and the split merge when rows are
+    split over several CTAs."""
+    ntiles = (k + 127) // 128
+    splits = max(1, min(16, ntiles, sms // max(T, 1)))
+    return 2 + (0 if streams else 1) + 1 + (1 if splits > 1 else 0)
+
+
 def rank_seed(cfg: int, rank: int) -> int:
     """Each rank draws its own replica batch (weak scaling)."""
     return cfg + 7919 * rank
@@ -263,19 +281,31 @@ def run_ours(args, rank, world, dist):
             clocks["note"] = "sampled during an equal-load loop right after the timed region (timed region too short)"
     ms_step = ms / args.steps
 
-    # ---- per-kernel breakdown: the same kernels through the component entry points
+    # ---- per-kernel breakdown: the same kernels dsa_forward runs, through the component
+    # entry points, with CUDA events between them on the launching stream
+    streams = forward_streams(T, max_n)
     nb = max(3, min(args.steps, 50))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
-    plan_ws = B.workspace(B.DSA_OP_INDEXER, T, max_n, k, device=dev)
     mla_ws = B.workspace(B.DSA_OP_SPARSE_MLA, T, max_n, k, device=dev)
-    ld = (max_n + 3) // 4 * 4
-    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    wm = work_model(n_vis_h, c.kv_start.cpu().numpy())
+    pk = peaks()
+    workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
+    if streams:
+        sel_ws = B.workspace(B.DSA_OP_INDEXER_TOPK, T, max_n, k, device=dev)
+    else:
+        plan_ws = B.workspace(B.DSA_OP_INDEXER, T, max_n, k, device=dev)
+        ld = (max_n + 3) // 4 * 4
+        scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
     torch.cuda.synchronize(dev)
     for e in evs:
         e[0].record(stream)
-        B.dsa_indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, scores, plan_ws, stream)
-        e[1].record(stream)
-        B.dsa_topk(scores, c.n_vis, k, idx, stream)
+        if streams:
+            B.dsa_indexer_topk(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, max_n, k, idx, sel_ws, stream)
+            e[1].record(stream)
+        else:
+            B.dsa_indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, scores, plan_ws, stream)
+            e[1].record(stream)
+            B.dsa_topk(scores, c.n_vis, k, idx, stream)
         e[2].record(stream)
         B.dsa_sparse_mla_attn(c.q, c.kv, c.kv_start, idx, wl.SCALE, o, lse, mla_ws, stream)
         e[3].record(stream)
@@ -284,19 +314,25 @@ def run_ours(args, rank, world, dist):
     t_idx = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_topk = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     t_att = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-
-    wm = work_model(n_vis_h, c.kv_start.cpu().numpy())
-    pk = peaks()
-    workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
-    per_kernel = {
-        "indexer": roofline_of("indexer (dsa_indexer_scores: plan + tcgen05 kernel)", t_idx, wm["indexer_bytes"],
-                               wm["indexer_flops"], pk, profiled_traffic("indexer", workload)),
-        "topk": roofline_of("top-k (dsa_topk)", t_topk, wm["topk_bytes"], 0.0, pk,
-                            profiled_traffic("topk", workload)),
-        "sparse_mla": roofline_of("sparse MLA (dsa_sparse_mla_attn: split CTAs + merge)", t_att,
-                                  wm["attention_bytes"], wm["attention_flops"], pk,
-                                  profiled_traffic("sparse_mla", workload)),
-    }
+    att = roofline_of("sparse MLA (dsa_sparse_mla_attn: split CTAs + merge)", t_att, wm["attention_bytes"],
+                      wm["attention_flops"], pk, profiled_traffic("sparse_mla", workload))
+    if streams:
+        sel_bytes = wm["indexer_bytes"] - 4 * float(n_vis_h.sum()) + 4 * k * T   # no score matrix, indices out
+        per_kernel = {
+            "indexer_topk": roofline_of("indexer + streamed top-k (dsa_indexer_topk: plan + tcgen05 kernel)",
+                                        t_idx, sel_bytes, wm["indexer_flops"], pk,
+                                        profiled_traffic("indexer_topk", workload)),
+            "sparse_mla": att,
+        }
+    else:
+        per_kernel = {
+            "indexer": roofline_of("indexer (dsa_indexer_scores: plan + tcgen05 kernel)", t_idx,
+                                   wm["indexer_bytes"], wm["indexer_flops"], pk,
+                                   profiled_traffic("indexer", workload)),
+            "topk": roofline_of("top-k (dsa_topk)", t_topk, wm["topk_bytes"], 0.0, pk,
+                                profiled_traffic("topk", workload)),
+            "sparse_mla": att,
+        }
     dominant = max(per_kernel, key=lambda kk: per_kernel[kk]["launch_ms"])
     roofline = per_kernel[dominant]
     kernels = {kk: {"ms": v["launch_ms"], "bound": v["bound"], "achieved": v["achieved"], "unit": v["unit"],
@@ -329,7 +365,8 @@ def run_ours(args, rank, world, dist):
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": launches_per_step(T, k, streams, torch.cuda.get_device_properties(dev).multi_processor_count)
+        * args.steps,
         "clocks": clocks,
     }
     if rank == 0:

@@ -78,7 +78,8 @@ enum dsa_op {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA = 2,
-  DSA_OP_FORWARD = 3
+  DSA_OP_FORWARD = 3,
+  DSA_OP_INDEXER_TOPK = 4
 };
 
 /*
@@ -151,6 +152,25 @@ DSA_API int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis
 DSA_API int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
                         const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,
                         size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Indexer and top-k fused, without a score matrix ("2026 LLM architecture
+ * overview (2): DSA and MoE of GLM 5 / DSV3.2", section 2.2: score every
+ * history position, keep index_topk of them).  Selects exactly what
+ * dsa_indexer_scores followed by dsa_topk selects, but each query's scores
+ * are filtered on the fly into a candidate buffer (kept in ws) that is cut
+ * back to the current top-k whenever it fills, so no T x n_vis matrix is
+ * written.  Rows of equal kv_start are processed together (up to 8), each
+ * group by one CTA over its whole context.
+ *
+ *  arguments as dsa_indexer_scores / dsa_topk; max_n_vis bounds n_vis
+ *  idx   [T,topk] int32: ascending positions, -1 padded (rows with invalid
+ *        n_vis / kv_start get all -1 and a status bit)
+ *  ws    >= dsa_workspace_size(DSA_OP_INDEXER_TOPK, T, max_n_vis, topk) bytes, 256-byte aligned
+ */
+DSA_API int dsa_indexer_topk(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                             const int64_t* kv_start, const int32_t* n_vis, int T, int64_t max_n_vis, int topk,
+                             int32_t* idx, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /*
  * The whole step: indexer -> top-k -> sparse MLA, enqueued on one stream.

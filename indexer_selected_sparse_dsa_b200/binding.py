@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_UNSUPPORTED, DSA_ERR_BAD_ROW = range(7)
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD = range(4)
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD, DSA_OP_INDEXER_TOPK = range(5)
 INDEX_HEADS, INDEX_DIM, HEADS, LATENT, ROPE, ROW, MAX_TOPK = 32, 128, 64, 512, 64, 576, 2048
 NOALLOC_MAX_ROWS = 8192
 
@@ -47,6 +47,8 @@ def lib():
         L.dsa_sparse_mla_attn.argtypes = [P, P, I64, P, P, I, I, F, P, P, P, SZ, P]
         L.dsa_forward.argtypes = [P, P, P, P, P, I64, P, P, I, I64, I, F, P, P, P, P, SZ, P]
         L.dsa_sync_status.argtypes = [P]
+        L.dsa_indexer_topk.argtypes = [P, P, P, I64, P, P, I, I64, I, P, P, SZ, P]
+        L.dsa_indexer_topk.restype = I
         L.dsa_indexer_scores_noalloc.argtypes = [P, P, P, I64, P, P, I, P, I64, P]
         L.dsa_indexer_scores_noalloc.restype = I
         L.dsa_last_error_string.restype = ctypes.c_char_p
@@ -121,6 +123,20 @@ def dsa_indexer_scores_noalloc(q_I, w, k_I, kv_start, n_vis, scores, stream=None
     _need(scores, torch.float32, None, "scores")
     _check(lib().dsa_indexer_scores_noalloc(_ptr(q_I), _ptr(w), _ptr(k_I), k_I.shape[0], _ptr(kv_start),
                                             _ptr(n_vis), T, _ptr(scores), scores.shape[1], _stream(stream)))
+
+
+def dsa_indexer_topk(q_I, w, k_I, kv_start, n_vis, max_n_vis, topk, idx, ws, stream=None):
+    import torch
+    T = n_vis.shape[0]
+    _need(q_I, torch.bfloat16, (T, INDEX_HEADS, INDEX_DIM), "q_I")
+    _need(w, torch.bfloat16, (T, INDEX_HEADS), "w")
+    _need(k_I, torch.bfloat16, None, "k_I")
+    _need(kv_start, torch.int64, (T,), "kv_start")
+    _need(n_vis, torch.int32, (T,), "n_vis")
+    _need(idx, torch.int32, (T, topk), "idx")
+    _need(ws, torch.uint8, None, "ws")
+    _check(lib().dsa_indexer_topk(_ptr(q_I), _ptr(w), _ptr(k_I), k_I.shape[0], _ptr(kv_start), _ptr(n_vis), T,
+                                  int(max_n_vis), topk, _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def dsa_topk(scores, n_vis, topk, idx, stream=None):

@@ -140,9 +140,24 @@ size_t ws_indexer(int T) { return align_up(dsa::indexer_plan_bytes(T), 256); }
 
 size_t ws_mla(int T, int topk) { return align_up(dsa::sparse_mla_part_bytes(T, dsa::sparse_mla_ws_splits(T, topk)), 256); }
 
+// dsa_forward streams scores into the selector (never stores them) when the score
+// matrix would be larger than this; DSA_FORWARD_MODE=stream|materialize overrides.
+constexpr size_t kStreamAboveBytes = size_t(8) << 30;
+
+bool forward_streams(int T, int64_t max_n_vis) {
+  if (const char* m = std::getenv("DSA_FORWARD_MODE")) {
+    if (!std::strcmp(m, "stream")) return true;
+    if (!std::strcmp(m, "materialize")) return false;
+  }
+  return size_t(T) * size_t(score_ld_for(max_n_vis)) * 4 > kStreamAboveBytes;
+}
+
+size_t ws_candidates(int T) { return align_up(size_t(T) * dsa::kStreamCap * 4, 256); }
+
 size_t ws_forward(int T, int64_t max_n_vis, int topk) {
-  return ws_indexer(T) + align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256) +
-         align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
+  const size_t sel = forward_streams(T, max_n_vis) ? 2 * ws_candidates(T)
+                                                   : align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256);
+  return ws_indexer(T) + sel + align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
 }
 
 int pick_qmax(int T) {
@@ -175,8 +190,8 @@ int run_sparse_mla(const dsa::MlaLaunch& p) {
 
 int run_indexer(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
                 const int64_t* kv_start, const int32_t* n_vis, int T, float* scores, int64_t score_ld, void* plan,
-                dsa_stream_t stream, int sm_count) {
-  int qmax = pick_qmax(T);
+                dsa_stream_t stream, int sm_count, const dsa::StreamOut* stream_out = nullptr) {
+  int qmax = stream_out ? 8 : pick_qmax(T);
   CUtensorMap tk, tq;
   int rc = make_tmap_bf16(&tk, k_I, DSA_INDEX_DIM, uint64_t(cache_rows), 128);
   if (rc) return rc;
@@ -201,6 +216,11 @@ int run_indexer(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int
   if (const char* sw = std::getenv("DSA_INDEXER_SWEEP")) {
     if (!std::strcmp(sw, "wave")) p.sweep = dsa::kSweepWave;
     if (!std::strcmp(sw, "split")) p.sweep = dsa::kSweepSplit;
+  }
+  p.streaming = stream_out != nullptr;
+  if (stream_out) {
+    p.stream_out = *stream_out;
+    p.sweep = dsa::kSweepWave;  // a CTA owns each query tile's whole sweep and its selection state
   }
   p.grid = sm_count;
   p.wait_ns = wait_limit_ns();
@@ -227,6 +247,7 @@ size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
     case DSA_OP_TOPK: return 0;
     case DSA_OP_SPARSE_MLA: return ws_mla(T, topk);
     case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
+    case DSA_OP_INDEXER_TOPK: return ws_indexer(T) + 2 * ws_candidates(T);
     default: return 0;
   }
 }
@@ -292,6 +313,35 @@ int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_row
   return run_sparse_mla(p);
 }
 
+int dsa_indexer_topk(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,
+                     const int64_t* kv_start, const int32_t* n_vis, int T, int64_t max_n_vis, int topk, int32_t* idx,
+                     void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
+  if (T == 0) return DSA_OK;
+  if (max_n_vis < 1 || max_n_vis > cache_rows)
+    return fail(DSA_ERR_INVALID_ARG, "max_n_vis must lie in [1, cache_rows]");
+  if (!q_I || !w || !k_I || !n_vis || !idx || !ws) return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_I, 16) || !aligned(w, 16) || !aligned(k_I, 16) || !aligned(n_vis, 4) || !aligned(idx, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q_I, w, k_I must be 16-byte aligned; n_vis, idx 4-byte aligned");
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (int64_t(T) * DSA_INDEX_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
+  const size_t need = ws_indexer(T) + 2 * ws_candidates(T);
+  if (ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, need);
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* sel = base + ws_indexer(T);
+  cudaError_t e = cudaMemsetAsync(idx, 0xFF, size_t(T) * size_t(topk) * 4, stream);  // rejected rows stay -1
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(idx)");
+  dsa::StreamOut so{reinterpret_cast<uint32_t*>(sel), reinterpret_cast<int32_t*>(sel + ws_candidates(T)), idx, topk,
+                    dsa::kStreamCap};
+  return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, nullptr, score_ld_for(max_n_vis), base, stream,
+                     dev->sm_count, &so);
+}
+
 int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q, const dsa_bf16* kv,
                 int64_t cache_rows, const int64_t* kv_start, const int32_t* n_vis, int T, int64_t max_n_vis, int topk,
                 float scale, float* o_lat, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes,
@@ -316,17 +366,32 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   if ((rc = current_device(&dev))) return rc;
 
   const int64_t ld = score_ld_for(max_n_vis);
+  const bool streams = forward_streams(T, max_n_vis);
   uint8_t* base = static_cast<uint8_t*>(ws);
   void* plan = base;
-  float* scores = reinterpret_cast<float*>(base + ws_indexer(T));
-  int32_t* idx_ws = reinterpret_cast<int32_t*>(base + ws_indexer(T) + align_up(size_t(T) * size_t(ld) * 4, 256));
+  uint8_t* sel = base + ws_indexer(T);  // score matrix, or the candidate buffers
+  const size_t sel_bytes = streams ? 2 * ws_candidates(T) : align_up(size_t(T) * size_t(ld) * 4, 256);
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(sel + sel_bytes);
   int32_t* idx = idx_out ? idx_out : idx_ws;
   float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(idx_ws) + align_up(size_t(T) * size_t(topk) * 4, 256));
 
-  if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, ld, plan, stream, dev->sm_count)))
-    return rc;
-  cudaError_t e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  cudaError_t e;
+  if (streams) {
+    // Rows the indexer plan rejects are never visited: they keep -1 everywhere.
+    if ((e = cudaMemsetAsync(idx, 0xFF, size_t(T) * size_t(topk) * 4, stream)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync(idx)");
+    dsa::StreamOut so{reinterpret_cast<uint32_t*>(sel), reinterpret_cast<int32_t*>(sel + ws_candidates(T)), idx,
+                      topk, dsa::kStreamCap};
+    if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, nullptr, ld, plan, stream, dev->sm_count,
+                          &so)))
+      return rc;
+  } else {
+    float* scores = reinterpret_cast<float*>(sel);
+    if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, ld, plan, stream, dev->sm_count)))
+      return rc;
+    e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  }
   dsa::MlaLaunch p{q,    kv,  cache_rows,        kv_start,      idx,           T,     topk, scale,
                    o_lat, lse, part,              ws_mla(T, topk), dev->sm_count, wait_limit_ns(), stream};
   return run_sparse_mla(p);

@@ -22,6 +22,7 @@
 #include <cuda.h>
 
 #include "block_scan.cuh"
+#include "group_select.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -183,15 +184,23 @@ struct UnitIter {
 // ------------------------------------------------------------------ main kernel
 constexpr int kEpiWarps = 8;
 constexpr int kIdxThreads = 64 + 32 * kEpiWarps;
+constexpr int kCheckUnits = 8;  // streaming selection: units between candidate-buffer checks
 
-template <int QMAX, int STAGES, int QBUF>
+template <int QMAX, int STAGES, int QBUF, bool STREAM>
 struct IdxSmem {
   static constexpr int kQBufBytes = QMAX * 2 * kQBoxBytes;  // two halves
   static constexpr int kKeysOff = 0;
   static constexpr int kQOff = STAGES * kStageBytes;
   static constexpr int kWOff = kQOff + QBUF * kQBufBytes;             // float w[QMAX*32]
   static constexpr int kNvOff = kWOff + QMAX * 32 * 4;                // int n_vis[QMAX]
-  static constexpr int kBarOff = (kNvOff + QMAX * 4 + 7) & ~7;
+  // streaming selection state: thresholds, counts, scan scratch, histogram, sort buffer
+  static constexpr int kThrOff = (kNvOff + QMAX * 4 + 15) & ~15;      // long long thr[QMAX]
+  static constexpr int kCntOff = kThrOff + QMAX * 8;                  // int cnt[QMAX]
+  static constexpr int kGsOff = kCntOff + QMAX * 4;                   // GroupShared
+  static constexpr int kHistOff = (kGsOff + int(sizeof(GroupShared)) + 15) & ~15;  // uint32 hist[4096]
+  static constexpr int kSortOff = kHistOff + 4096 * 4;                // int sort[2048]
+  static constexpr int kStreamEnd = STREAM ? kSortOff + 2048 * 4 : kNvOff + QMAX * 4;
+  static constexpr int kBarOff = (kStreamEnd + 7) & ~7;
   static constexpr int kNumBars = 2 * STAGES + 2 * QBUF + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;             // tmem slot, abort flag
   static constexpr int kBytes = kMiscOff + 16;
@@ -200,13 +209,13 @@ struct IdxSmem {
   static constexpr int kTmemCols = (2 * kAccCols) <= 32 ? 32 : (2 * kAccCols);
 };
 
-template <int QMAX, int STAGES, int QBUF>
+template <int QMAX, int STAGES, int QBUF, bool STREAM>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const uint16_t* __restrict__ w, const int32_t* __restrict__ n_vis,
                    const PlanHeader* __restrict__ hdr, const PlanTile* __restrict__ tiles, float* __restrict__ scores,
-                   int64_t score_ld, int sweep, WaitLimit lim) {
-  using L = IdxSmem<QMAX, STAGES, QBUF>;
+                   int64_t score_ld, int sweep, StreamOut so, WaitLimit lim) {
+  using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -352,6 +361,58 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int half = (warp - 2) >> 2;     // queries half, half + 2, half + 4, ...
     const int row = quarter * 32 + lane;
     const int et = threadIdx.x - 64;      // 0 .. 32 * kEpiWarps - 1
+    long long* thr_s = reinterpret_cast<long long*>(smem + L::kThrOff);
+    int* cnt_s = reinterpret_cast<int*>(smem + L::kCntOff);
+    GroupShared& gs = *reinterpret_cast<GroupShared*>(smem + L::kGsOff);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
+    int* sortbuf = reinterpret_cast<int*>(smem + L::kSortOff);
+    // Keep the topk best entries of query q's buffer (exact: ties at the cut go to the
+    // lowest positions), move them to its front and raise its filter threshold.
+    auto stream_shrink = [&](int q, int q0, const Group& g) {
+      const long long ro = (long long)(q0 + q) * so.cap;
+      const int m = min(cnt_s[q], so.cap);
+      if (m <= so.topk) return;
+      const uint32_t* ck = so.cand_key + ro;
+      int32_t* cp = so.cand_pos + ro;
+      const Rule r = group_radix_select(m, so.topk, hist, gs, g, [&](int j) { return ck[j]; },
+                                        [](int) { return true; });
+      long long cut = 0;  // among keys == r.thr keep positions p with ~p >= cut
+      if (r.keep_eq > 0) {
+        const Rule rp = group_radix_select(
+            m, r.keep_eq, hist, gs, g, [&](int j) { return ~uint32_t(cp[j]); },
+            [&](int j) { return (long long)ck[j] == r.thr; });
+        cut = rp.keep_eq > 0 ? rp.thr : rp.thr + 1;
+      }
+      const int kept = group_compact(
+          m, gs, g, [&](int j) { return make_uint2(ck[j], uint32_t(cp[j])); },
+          [&](uint2 e) {
+            const long long k = e.x;
+            return k > r.thr || (r.keep_eq > 0 && k == r.thr && (long long)(~e.y) >= cut);
+          },
+          [&](int dst, uint2 e) {
+            so.cand_key[ro + dst] = e.x;
+            so.cand_pos[ro + dst] = int32_t(e.y);
+          });
+      if (g.tid == 0) {
+        cnt_s[q] = kept;
+        thr_s[q] = r.thr;
+      }
+      g.sync();
+    };
+    // Final selection of query q: its kept positions, ascending, padded with -1.
+    auto stream_finish = [&](int q, int q0, const Group& g) {
+      stream_shrink(q, q0, g);
+      const long long ro = (long long)(q0 + q) * so.cap;
+      const int m = min(cnt_s[q], so.topk);
+      int np2 = 1;
+      while (np2 < m) np2 <<= 1;
+      for (int j = g.tid; j < np2; j += g.n) sortbuf[j] = j < m ? so.cand_pos[ro + j] : 0x7fffffff;
+      g.sync();
+      group_bitonic_sort(sortbuf, np2, g);
+      int32_t* out = so.idx + (long long)(q0 + q) * so.topk;
+      for (int j = g.tid; j < so.topk; j += g.n) out[j] = j < m ? sortbuf[j] : -1;
+      g.sync();
+    };
     UnitIter it;
     it.sweep = sweep;
     int prev_tile = -1, ab = 0;
@@ -364,6 +425,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         for (int e = et; e < nq * 32; e += 32 * kEpiWarps)
           w_s[e] = bf16_bits_to_float(w[(long long)it.cur.q0 * 32 + e]);
         if (et < nq) nv_s[et] = n_vis[it.cur.q0 + et];
+        if constexpr (STREAM) {
+          if (et < QMAX) {
+            thr_s[et] = -1;  // nothing kept yet: every score passes
+            cnt_s[et] = 0;
+          }
+        }
         named_bar_sync(1, 32 * kEpiWarps);
         prev_tile = it.tile;
       }
@@ -371,6 +438,29 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       tc_fence_after();
       const long long s = (long long)it.kt * kKeysPerUnit + row;
       const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
+      // score of (query qi, key s): written out, or offered to the query's candidate buffer
+      auto emit = [&](int qi, float score) {
+        const bool in = s < nv_s[qi];
+        if constexpr (!STREAM) {
+          if (in) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = score;
+        } else {
+          const uint32_t key = float_order_key(score);
+          const bool pass = in && (long long)key > thr_s[qi];
+          const unsigned m = __ballot_sync(0xffffffffu, pass);
+          if (m) {
+            const int leader = __ffs(m) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&cnt_s[qi], __popc(m));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const int off = base + __popc(m & ((1u << lane) - 1u));
+            if (pass && off < so.cap) {
+              const long long ro = (long long)(it.cur.q0 + qi) * so.cap;
+              so.cand_key[ro + off] = key;
+              so.cand_pos[ro + off] = int(s);
+            }
+          }
+        }
+      };
       // this warp's queries, two per TMEM wait: qi = half, half + 2 (then + 4, + 6)
       for (int qi = half; qi < nq; qi += 4) {
         const int qj = qi + 2;
@@ -390,7 +480,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           a0 = fmaf(c.z, v[4 * h4 + 2], a0);
           a0 = fmaf(c.w, v[4 * h4 + 3], a0);
         }
-        if (s < nv_s[qi]) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = a0;
+        emit(qi, a0);
         if (qj < nq) {
           const float4* w1 = reinterpret_cast<const float4*>(w_s + qj * 32);
 #pragma unroll
@@ -401,12 +491,26 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             a1 = fmaf(c.z, v[32 + 4 * h4 + 2], a1);
             a1 = fmaf(c.w, v[32 + 4 * h4 + 3], a1);
           }
-          if (s < nv_s[qj]) scores[(long long)(it.cur.q0 + qj) * score_ld + s] = a1;
+          emit(qj, a1);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(aempty_bar(ab));
+      if constexpr (STREAM) {
+        // Every kCheckUnits units: shrink buffers that could overflow before the next
+        // check (a query gains at most one entry per key); after the tile's last unit,
+        // finish its queries.
+        const bool last = it.kt == it.cur.units - 1;
+        if (last || (it.kt % kCheckUnits) == kCheckUnits - 1) {
+          const Group g{et, 32 * kEpiWarps, 1};
+          g.sync();
+          for (int q = 0; q < nq; ++q)
+            if (cnt_s[q] > so.cap - kCheckUnits * kKeysPerUnit) stream_shrink(q, it.cur.q0, g);
+          if (last)
+            for (int q = 0; q < nq; ++q) stream_finish(q, it.cur.q0, g);
+        }
+      }
       if (++ab == 2) {
         ab = 0;
         aphase ^= 1u;
@@ -424,21 +528,21 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   }
 }
 
-template <int QMAX, int STAGES, int QBUF>
+template <int QMAX, int STAGES, int QBUF, bool STREAM>
 cudaError_t set_smem_attr() {
-  using L = IdxSmem<QMAX, STAGES, QBUF>;
+  using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
   static_assert(L::kAlloc <= 232448, "indexer shared memory exceeds the per-CTA limit");
-  return cudaFuncSetAttribute(indexer_kernel<QMAX, STAGES, QBUF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              L::kAlloc);
+  return cudaFuncSetAttribute(indexer_kernel<QMAX, STAGES, QBUF, STREAM>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
 }
 
-template <int QMAX, int STAGES, int QBUF>
+template <int QMAX, int STAGES, int QBUF, bool STREAM>
 cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUtensorMap& tq) {
-  using L = IdxSmem<QMAX, STAGES, QBUF>;
+  using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
   auto* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<const PlanTile*>(reinterpret_cast<const uint8_t*>(p.plan) + sizeof(PlanHeader));
-  indexer_kernel<QMAX, STAGES, QBUF><<<p.grid, kIdxThreads, L::kAlloc, p.stream>>>(
-      tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, WaitLimit{p.wait_ns});
+  indexer_kernel<QMAX, STAGES, QBUF, STREAM><<<p.grid, kIdxThreads, L::kAlloc, p.stream>>>(
+      tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, p.stream_out, WaitLimit{p.wait_ns});
   return cudaGetLastError();
 }
 
@@ -446,9 +550,10 @@ cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUt
 
 cudaError_t prepare_indexer() {
   cudaError_t e;
-  if ((e = set_smem_attr<1, 6, 2>()) != cudaSuccess) return e;
-  if ((e = set_smem_attr<4, 4, 2>()) != cudaSuccess) return e;
-  if ((e = set_smem_attr<8, 4, 1>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<1, 6, 2, false>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<4, 4, 2, false>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<8, 4, 1, false>()) != cudaSuccess) return e;
+  if ((e = set_smem_attr<8, 4, 1, true>()) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -460,10 +565,11 @@ cudaError_t launch_indexer(const IndexerLaunch& p, const CUtensorMap& tmap_k, co
                                                 tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.streaming) return p.qmax == 8 ? launch_main<8, 4, 1, true>(p, tmap_k, tmap_q) : cudaErrorInvalidValue;
   switch (p.qmax) {
-    case 1: return launch_main<1, 6, 2>(p, tmap_k, tmap_q);
-    case 4: return launch_main<4, 4, 2>(p, tmap_k, tmap_q);
-    case 8: return launch_main<8, 4, 1>(p, tmap_k, tmap_q);
+    case 1: return launch_main<1, 6, 2, false>(p, tmap_k, tmap_q);
+    case 4: return launch_main<4, 4, 2, false>(p, tmap_k, tmap_q);
+    case 8: return launch_main<8, 4, 1, false>(p, tmap_k, tmap_q);
     default: return cudaErrorInvalidValue;
   }
 }

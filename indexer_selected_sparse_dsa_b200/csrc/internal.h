@@ -35,6 +35,17 @@ enum SweepMode : int {
   kSweepWave = 1,   // CTA c takes whole query tiles c, c+G, ... (shared-key L2 reuse)
 };
 
+// Streaming selection (no score matrix): per query row a candidate buffer of
+// `cap` (order key, position) pairs; the kept positions go to idx[T, topk].
+struct StreamOut {
+  uint32_t* cand_key;  // [T, cap]
+  int32_t* cand_pos;   // [T, cap]
+  int32_t* idx;        // [T, topk]
+  int topk;
+  int cap;
+};
+constexpr int kStreamCap = 8192;
+
 struct IndexerLaunch {
   const uint16_t* q_I;
   const uint16_t* w;
@@ -48,6 +59,8 @@ struct IndexerLaunch {
   void* plan;  // indexer_plan_bytes(T) bytes
   int qmax;    // 1, 4 or 8
   int sweep;   // SweepMode
+  bool streaming;  // select into stream_out instead of writing scores (wave sweep, qmax 8)
+  StreamOut stream_out;
   int grid;    // persistent CTAs
   unsigned long long wait_ns;
   cudaStream_t stream;

@@ -510,34 +510,48 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
 // Merge the splits of each query row: with M = max_s m_s,
 //   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 of the denominator) * ln 2.
-__global__ void __launch_bounds__(512) sparse_mla_combine_kernel(const float* __restrict__ part, int splits,
-                                                                 float* __restrict__ o_lat,
-                                                                 float* __restrict__ lse) {
-  __shared__ float wgt[16][64];
-  __shared__ float inv_den[64];
-  const int i = blockIdx.x;
+// One CTA per (row, group of 4 heads): 2048 outputs, float4 loads of every split in flight.
+constexpr int kCombineHeads = 4;
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads) sparse_mla_combine_kernel(const float* __restrict__ part,
+                                                                             int splits, float* __restrict__ o_lat,
+                                                                             float* __restrict__ lse) {
+  __shared__ float wgt[16][kCombineHeads];
+  __shared__ float inv_den[kCombineHeads];
+  const int groups = 64 / kCombineHeads;
+  const int i = blockIdx.x / groups;
+  const int h0 = (blockIdx.x - i * groups) * kCombineHeads;
   const float* p = part + (long long)i * splits * kPartFloats;
-  if (threadIdx.x < 64) {
-    const int h = threadIdx.x;
+  if (threadIdx.x < kCombineHeads) {
+    const int h = h0 + threadIdx.x;
     float M = -INFINITY;
     for (int s = 0; s < splits; ++s) M = fmax_(M, p[(long long)s * kPartFloats + 64 * 512 + h]);
     float den = 0.f;
     for (int s = 0; s < splits; ++s) {
       const float ms = p[(long long)s * kPartFloats + 64 * 512 + h];
       const float w = (M == -INFINITY) ? 0.f : fast_exp2(ms - M);
-      wgt[s][h] = w;
+      wgt[s][threadIdx.x] = w;
       den += w * p[(long long)s * kPartFloats + 64 * 512 + 64 + h];
     }
-    inv_den[h] = den > 0.f ? 1.f / den : 0.f;
+    inv_den[threadIdx.x] = den > 0.f ? 1.f / den : 0.f;
     if (lse) lse[(long long)i * 64 + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
+  const long long base = (long long)h0 * 512;
   float* orow = o_lat + (long long)i * 64 * 512;
-  for (int e = threadIdx.x; e < 64 * 512; e += blockDim.x) {
-    const int h = e >> 9;
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s) acc += wgt[s][h] * p[(long long)s * kPartFloats + e];
-    orow[e] = acc * inv_den[h];
+  for (int v = threadIdx.x; v < kCombineHeads * 512 / 4; v += kCombineThreads) {
+    const int hl = (v * 4) >> 9;  // head within the group
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+      const float4 x = *reinterpret_cast<const float4*>(p + (long long)s * kPartFloats + base + v * 4);
+      const float w = wgt[s][hl];
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
+    }
+    const float id = inv_den[hl];
+    *reinterpret_cast<float4*>(orow + base + v * 4) = make_float4(acc.x * id, acc.y * id, acc.z * id, acc.w * id);
   }
 }
 
@@ -573,7 +587,8 @@ cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q) {
       WaitLimit{p.wait_ns});
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
-  sparse_mla_combine_kernel<<<p.T, 512, 0, p.stream>>>(p.part, splits, p.o_lat, p.lse);
+  sparse_mla_combine_kernel<<<p.T * (64 / kCombineHeads), kCombineThreads, 0, p.stream>>>(p.part, splits, p.o_lat,
+                                                                                         p.lse);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,14 @@ __device__ void find_bin(int nb, int need, TopkShared& sh) {
   __syncthreads();
 }
 
+// Add 1 to hist[bin] for every calling lane; lanes of a warp with equal bins add
+// once (candidate keys crowd into a few bins, where plain atomics serialise).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
+  const unsigned mask = __activemask();
+  const unsigned peers = __match_any_sync(mask, bin);
+  if ((threadIdx.x & 31) == unsigned(__ffs(peers) - 1)) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
+}
+
 // Radix selection of the `need`-th largest of m keys, 12 + 10 + 10 bits;
 // key(j) reads key j.
 template <class Key>
@@ -103,7 +111,7 @@ __device__ KeepRule radix_select(int m, int need, TopkShared& sh, Key key) {
     __syncthreads();
     for (int j = threadIdx.x; j < m; j += blockDim.x) {
       const uint32_t k = key(j);
-      if (bits_done == 0 || (k >> (32 - bits_done)) == prefix) atomicAdd(&sh.hist[(k >> shift) & uint32_t(nb - 1)], 1u);
+      if (bits_done == 0 || (k >> (32 - bits_done)) == prefix) hist_add(sh.hist, (k >> shift) & uint32_t(nb - 1));
     }
     __syncthreads();
     find_bin(nb, need, sh);
@@ -203,14 +211,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
     const int per_iter = int(blockDim.x) * kVec * 4;
     const int n_main = (n / per_iter) * per_iter;
     int total = 0;
+    // the next iteration's loads are issued before this one is compacted
+    float4 nxt[kVec];
+    if (n_main > 0) {
+      const float4* p4 = reinterpret_cast<const float4*>(row + int(threadIdx.x) * kVec * 4);
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) nxt[u] = __ldg(p4 + u);
+    }
     for (int base = 0; base < n; base += per_iter) {
       uint32_t keys[kVec * 4];
       const int j0 = base + int(threadIdx.x) * kVec * 4;  // this thread's 32 consecutive positions
       if (base < n_main) {
-        const float4* p4 = reinterpret_cast<const float4*>(row + j0);
         float4 v[kVec];
 #pragma unroll
-        for (int u = 0; u < kVec; ++u) v[u] = __ldg(p4 + u);
+        for (int u = 0; u < kVec; ++u) v[u] = nxt[u];
+        if (base + per_iter < n_main) {
+          const float4* p4 = reinterpret_cast<const float4*>(row + j0 + per_iter);
+#pragma unroll
+          for (int u = 0; u < kVec; ++u) nxt[u] = __ldg(p4 + u);
+        }
 #pragma unroll
         for (int u = 0; u < kVec; ++u) {
           keys[4 * u] = order_key(v[u].x);

@@ -127,12 +127,16 @@ def host_rows(c, rows):
     nv = c.n_vis.cpu().numpy()
     kI, kv, starts = [], [], []
     off = 0
+    seen = {}   # rows of one sequence share one copy of its prefix
     for r in rows:
-        s0, n = int(ks[r]), int(nv[r])
-        kI.append(u16(c.k_I[s0:s0 + n]))
-        kv.append(u16(c.kv[s0:s0 + n]))
-        starts.append(off)
-        off += n
+        s0 = int(ks[r])
+        n = int(max(nv[q] for q in rows if int(ks[q]) == s0))
+        if s0 not in seen:
+            kI.append(u16(c.k_I[s0:s0 + n]))
+            kv.append(u16(c.kv[s0:s0 + n]))
+            seen[s0] = off
+            off += n
+        starts.append(seen[s0])
     return dict(q_I=u16(c.q_I[rows]), w=u16(c.w[rows]), q=u16(c.q[rows]), k_I=np.concatenate(kI),
                 kv=np.concatenate(kv), kv_start=np.array(starts, np.int64), n_vis=nv[rows].astype(np.int32),
                 plants=c.plants[rows])

@@ -274,3 +274,67 @@ def test_forward_causal_prefill_short_rows():
 
 def test_forward_ragged_decode_scaled():
     _forward_check(wl.make_workload_numpy(3, scale=32))
+
+
+# ---------------------------------------------------------------------------- streamed selection
+
+STREAM_CASES = {
+    # the query tile's candidate buffers shrink several times (rows much longer than 8192)
+    "long_shared": lambda: wl.make_case_numpy([30000], [(0, 30000), (0, 29999), (0, 25000), (0, 9000), (0, 2048),
+                                                        (0, 2049), (0, 100), (0, 1)], seed=61),
+    "scaled_chunked_prefill": lambda: wl.make_workload_numpy(4, scale=64),
+    "mixed_sequences": lambda: wl.make_case_numpy([20000, 5000, 12000], [(0, 20000), (1, 5000), (2, 12000),
+                                                                          (2, 11000), (0, 19999)], seed=62),
+}
+
+
+@pytest.mark.parametrize("name", sorted(STREAM_CASES))
+def test_forward_streamed_selection_equals_materialized(name, monkeypatch):
+    c = STREAM_CASES[name]()
+    d = to_dev(c)
+    maxn = int(max(c.n_vis))
+    monkeypatch.setenv("DSA_FORWARD_MODE", "materialize")
+    o_m, lse_m, idx_m = gpu_forward(d, maxn, 2048)
+    monkeypatch.setenv("DSA_FORWARD_MODE", "stream")
+    o_s, lse_s, idx_s = gpu_forward(d, maxn, 2048)
+    assert np.array_equal(idx_m, idx_s)
+    assert np.array_equal(o_m, o_s) and np.array_equal(lse_m, lse_s)
+    S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=maxn)
+    assert_selection_ok(idx_s, S_ref, c.n_vis, 2048)
+    for i in range(c.T):
+        p = c.plants[i][c.plants[i] >= 0]
+        assert np.isin(p, idx_s[i]).all()
+
+
+def test_forward_streamed_ties_go_to_lowest_positions(monkeypatch):
+    # keys of the second sequence are all zero: every score is exactly 0, so the
+    # selection must be positions 0..2047 in both modes
+    c = wl.make_case_numpy([12000, 15000], [(0, 12000), (1, 15000), (1, 9000)], seed=63, n_plant=0)
+    c.k_I[12000:] = 0
+    d = to_dev(c)
+    monkeypatch.setenv("DSA_FORWARD_MODE", "stream")
+    _, _, idx = gpu_forward(d, 15000, 2048)
+    assert idx[1].tolist() == list(range(2048)) and idx[2].tolist() == list(range(2048))
+    monkeypatch.setenv("DSA_FORWARD_MODE", "materialize")
+    _, _, idx_m = gpu_forward(d, 15000, 2048)
+    assert np.array_equal(idx, idx_m)
+
+
+@pytest.mark.parametrize("name", sorted(STREAM_CASES))
+def test_indexer_topk_equals_scores_then_topk(name):
+    """The fused entry point selects exactly what dsa_indexer_scores + dsa_topk select."""
+    import torch
+    c = STREAM_CASES[name]()
+    d = to_dev(c)
+    T, maxn, k = c.T, int(max(c.n_vis)), 2048
+    ld = (maxn + 3) // 4 * 4
+    scores = torch.empty((T, ld), dtype=torch.float32, device="cuda")
+    B.dsa_indexer_scores(d["q_I"], d["w"], d["k_I"], d["kv_start"], d["n_vis"], scores,
+                         B.workspace(B.DSA_OP_INDEXER, T, ld, 0))
+    idx_a = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    B.dsa_topk(scores, d["n_vis"], k, idx_a)
+    idx_b = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    B.dsa_indexer_topk(d["q_I"], d["w"], d["k_I"], d["kv_start"], d["n_vis"], maxn, k, idx_b,
+                       B.workspace(B.DSA_OP_INDEXER_TOPK, T, maxn, k))
+    B.dsa_sync_status()
+    assert np.array_equal(idx_a.cpu().numpy(), idx_b.cpu().numpy())
