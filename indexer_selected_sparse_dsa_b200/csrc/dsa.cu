@@ -287,7 +287,7 @@ int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T,
   DeviceState* dev = nullptr;
   int rc = current_device(&dev);
   if (rc) return rc;
-  cudaError_t e = dsa::launch_topk(scores, score_ld, n_vis, T, topk, idx, stream);
+  cudaError_t e = dsa::launch_topk(scores, score_ld, n_vis, T, topk, idx, dev->sm_count, stream);
   if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
   return DSA_OK;
 }
@@ -389,7 +389,7 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
     float* scores = reinterpret_cast<float*>(sel);
     if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, ld, plan, stream, dev->sm_count)))
       return rc;
-    e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, stream);
+    e = dsa::launch_topk(scores, ld, n_vis, T, topk, idx, dev->sm_count, stream);
     if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
   }
   dsa::MlaLaunch p{q,    kv,  cache_rows,        kv_start,      idx,           T,     topk, scale,

@@ -80,12 +80,7 @@ __device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared&
     for (int j = g.tid; j < m; j += g.n) {
       if (!inc(j)) continue;
       const uint32_t k = key(j);
-      if (bits_done == 0 || (k >> (32 - bits_done)) == prefix) {
-        // lanes of a warp with equal bins add once: candidates crowd into few bins
-        const uint32_t bin = (k >> shift) & uint32_t(nb - 1);
-        const unsigned peers = __match_any_sync(__activemask(), bin);
-        if ((g.tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
-      }
+      if (bits_done == 0 || (k >> (32 - bits_done)) == prefix) atomicAdd(&hist[(k >> shift) & uint32_t(nb - 1)], 1u);
     }
     g.sync();
     // bin where the count from the top first reaches `need`

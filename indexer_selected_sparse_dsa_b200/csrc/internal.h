@@ -68,8 +68,10 @@ struct IndexerLaunch {
 cudaError_t launch_indexer(const IndexerLaunch& p, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q);
 
 // ------------------------------------------------------------------ top-k
+// Rows longer than a few chunks are split over a cluster of up to 4 CTAs when
+// there are fewer rows than SMs.
 cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk,
-                        int32_t* idx, cudaStream_t stream);
+                        int32_t* idx, int sm_count, cudaStream_t stream);
 
 // ------------------------------------------------------------------ sparse MLA
 struct MlaLaunch {

@@ -104,7 +104,11 @@ def _topk_case(kind, n, seed):
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "wide"])
 @pytest.mark.parametrize("k", [1, 7, 2048])
-def test_topk_bit_exact(kind, k):
+@pytest.mark.parametrize("split", [None, "4"])
+def test_topk_bit_exact(kind, k, split, monkeypatch):
+    # split "4": every row over a cluster of 4 CTAs (a 20000-key row leaves one idle)
+    if split:
+        monkeypatch.setenv("DSA_TOPK_SPLIT", split)
     lens = [1, 5, k - 1 if k > 1 else 1, k, k + 1, 2047, 2049, 5000, 20000]
     ld = (max(lens) + 3) // 4 * 4
     S = np.full((len(lens), ld), np.nan, np.float32)
@@ -117,8 +121,10 @@ def test_topk_bit_exact(kind, k):
         assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
 
 
-@pytest.mark.parametrize("path", ["filtered", "full"])
-def test_topk_long_rows_exact(path, monkeypatch):
+@pytest.mark.parametrize("path,split", [("filtered", "1"), ("filtered", "2"), ("filtered", "4"), ("full", "1"),
+                                        ("full", "2")])
+def test_topk_long_rows_exact(path, split, monkeypatch):
+    monkeypatch.setenv("DSA_TOPK_SPLIT", split)
     if path == "full":
         monkeypatch.setenv("DSA_TOPK_KERNEL", "row")
     lens = [131072, 204800, 65537]
@@ -131,7 +137,9 @@ def test_topk_long_rows_exact(path, monkeypatch):
     assert np.array_equal(gpu_topk(S, n_vis, 2048), ref)
 
 
-def test_topk_filter_fallbacks():
+@pytest.mark.parametrize("split", ["1", "4"])
+def test_topk_filter_fallbacks(split, monkeypatch):
+    monkeypatch.setenv("DSA_TOPK_SPLIT", split)
     # rows where the sample threshold admits too many keys (all equal, sorted
     # ascending with a constant tail) or where the sample misses the top keys
     n, k = 50000, 2048
@@ -146,6 +154,31 @@ def test_topk_filter_fallbacks():
     n_vis = np.full(4, n, np.int32)
     ref = oracle.topk(S.astype(np.float64), n_vis, k)
     assert np.array_equal(gpu_topk(S, n_vis, k), ref)
+
+
+@pytest.mark.parametrize("k", [7, 2048])
+@pytest.mark.parametrize("split", ["1", "2", "4"])
+def test_topk_buffer_cuts_exact(k, split, monkeypatch):
+    monkeypatch.setenv("DSA_TOPK_SPLIT", split)
+    # rows whose candidates overflow the on-chip buffer while streaming, so it
+    # is cut to its exact top-k (ties to lower positions) one or more times
+    n = 300000
+    r = np.random.default_rng(11 + k)
+    rows = [
+        np.arange(n, dtype=np.float32),                                   # every chunk beats the last
+        np.full(n, 2.5, np.float32),                                      # one tie class
+        (np.arange(n) // 1000).astype(np.float32),                        # ascending plateaus of ties
+        (np.arange(n) * 1e-4 + r.standard_normal(n)).astype(np.float32),  # drift plus noise
+        np.where(np.arange(n) % 3 == 0, 1.0, 0.0).astype(np.float32),     # comb of ties
+        r.integers(0, 3, n).astype(np.float32),                           # three tie classes
+    ]
+    S = np.stack(rows)
+    n_vis = np.full(len(rows), n, np.int32)
+    n_vis[4] = n - 5                                                      # ragged tail
+    ref = oracle.topk(S.astype(np.float64), n_vis, k)
+    got = gpu_topk(S, n_vis, k)
+    for i in range(len(rows)):
+        assert np.array_equal(got[i], ref[i]), f"row {i}"
 
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "wide"])
