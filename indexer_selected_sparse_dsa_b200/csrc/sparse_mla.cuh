@@ -14,8 +14,9 @@
 //    selected rows in the 128-byte-swizzled layout the tensor cores read,
 //    filled with 16-byte cp.async (an empty index slot is zero-filled); each
 //    thread's copies arrive on the slot's mbarrier when they land, so every
-//    free slot of the ring is in flight; the rows of tile t+1 are prefetched
-//    into L2 while tile t is staged.  Per tile t the stream
+//    free slot of the ring is in flight; the selected positions are read two
+//    tiles ahead.  (An L2 prefetch of the next tile's rows measured slower:
+//    the bulk prefetches queue ahead of the copies.)  Per tile t the stream
 //    carries its key chunks 0..8 (five slots) and, one tile later, its latent
 //    chunks 0..7 again (four slots) for the value product: the rows cross L2
 //    twice instead of holding a 144 KB tile.
@@ -23,10 +24,13 @@
 //    K = 576) into one of two TMEM buffers, one tile ahead of
 //    O^T += V_t^T . P_t^T (M = 128 latent dims x 4, N = 64, K = 128), with V
 //    read MN-major straight from the slot.
-//  * warps 5..8, softmax: each thread owns one key row of S^T; fp32 running
-//    max and sum per head (62-shuffle reduce-scatter per warp + 4-way combine),
-//    lazy rescale of O when a tile max passes the running max by 2^8; P goes
-//    to shared memory as bf16 for the value product.
+//  * warps 5..8, softmax: each thread owns one key row of S^T.  Exponents are
+//    taken against a lazily updated running max: each thread checks its own
+//    row against it, and only when some score passes it by 2^8 (one barrier
+//    vote) is the tile max reduced across the CTA and O rescaled.  Each thread
+//    keeps its row's share of the running sums in registers; they are reduced
+//    once after the last tile.  P goes to shared memory as bf16 for the value
+//    product.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -254,27 +258,26 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
       return true;
     };
+    // Selected positions run two tiles ahead in registers (one key row per
+    // thread), so staging a tile never waits on a global load.
+    auto load_pos = [&](int tile) {
+      const int slot_i = (t_first + tile) * kTileKeys + pt;
+      return (tile < ntiles && slot_i < topk) ? irow[slot_i] : -1;
+    };
+    int v0 = load_pos(0), v1 = load_pos(1);
     for (int s = 0; s <= ntiles && ok; ++s) {
       if (s < ntiles) {
         // cache rows of tile s (-1: empty or out of range) into y_s[s & 1]
         named_bar_sync(2, 128);  // every producer is done reading this buffer's previous tile
         {
-          const int slot_i = (t_first + s) * kTileKeys + pt;
           int yy = -1;
-          if (slot_i < topk) {
-            const int v = irow[slot_i];
-            if (v >= 0) {
-              if (ks + v < cache_rows) yy = int(ks + v);
-              else raise_status(kStatusBadRow);
-            }
+          if (v0 >= 0) {
+            if (ks + v0 < cache_rows) yy = int(ks + v0);
+            else raise_status(kStatusBadRow);
           }
           y_s[(s & 1) * 128 + pt] = yy;
-          // pull the next tile's rows into L2 now, so its slot loads are L2 hits
-          const int slot_n = slot_i + kTileKeys;
-          if (s + 1 < ntiles && slot_n < topk) {
-            const int v = irow[slot_n];
-            if (v >= 0 && ks + v < cache_rows) prefetch_l2_bulk(kv + (ks + v) * kRow, kRow * 2);
-          }
+          v0 = v1;
+          v1 = load_pos(s + 2);
         }
         named_bar_sync(2, 128);
         cur_skip = 0u;
@@ -369,6 +372,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const int r = quarter * 32 + lane;
     const int rw = st >> 5;           // slot of this warp in red[]
     const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    // This thread's share of each head's running sum (its key row over all
+    // tiles); reduced across the 128 threads once, after the last tile.
+    float l_acc[64];
+#pragma unroll
+    for (int h = 0; h < 64; ++h) l_acc[h] = 0.f;
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
       const int slot_i = (t_first + t) * kTileKeys + r;
@@ -379,32 +387,43 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
       if (!(ok = mbar_wait(s_full(t & 1), uint32_t((t >> 1) & 1), lim, abort_flag))) break;
       tc_fence_after();
-      float x[64];
-      tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1), x);
-      tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1) + 32, x + 32);
+      // Lazy running max: exponents stay taken against m_use while no score of
+      // the tile passes it by more than 2^kLazyRescale, which each thread checks
+      // for its own key row; only then is the tile max reduced and O rescaled.
+      int above = 0;
 #pragma unroll
-      for (int h = 0; h < 64; ++h) x[h] = valid ? x[h] * scale_log2 : -INFINITY;
-
-      // per-head max over the tile's 128 keys
-      float r0, r1;
-      reduce_scatter64<true>(x, r0, r1);
-      red[rw * 64 + 2 * lane] = r0;
-      red[rw * 64 + 2 * lane + 1] = r1;
-      named_bar_sync(1, 128);
-      int resc = 0;
-      if (st < 64) {
-        const float mt = fmax_(fmax_(red[st], red[64 + st]), fmax_(red[128 + st], red[192 + st]));
-        const float mu = m_use[st];
-        float al = 1.f;
-        if (mt > -INFINITY && (mu == -INFINITY || mt > mu + kLazyRescale)) {
-          al = fast_exp2(mu - mt);  // 0 when mu = -inf
-          m_use[st] = mt;
-          l_run[st] *= al;
-          resc = (t > 0) && (al != 1.f);
-        }
-        alpha_s[st] = al;
+      for (int half = 0; half < 2; ++half) {
+        float y[32];
+        tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1) + 32 * half, y);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) above |= (valid && y[h] * scale_log2 > m_use[32 * half + h] + kLazyRescale) ? 1 : 0;
       }
-      resc = bar_red_or_128(resc);  // also the barrier that publishes m_use / alpha
+      int resc = 0;
+      if (bar_red_or_128(above)) {
+        float x[64];
+        tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1), x);
+        tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1) + 32, x + 32);
+#pragma unroll
+        for (int h = 0; h < 64; ++h) x[h] = valid ? x[h] * scale_log2 : -INFINITY;
+        float r0, r1;
+        reduce_scatter64<true>(x, r0, r1);
+        red[rw * 64 + 2 * lane] = r0;
+        red[rw * 64 + 2 * lane + 1] = r1;
+        named_bar_sync(1, 128);
+        int mine = 0;
+        if (st < 64) {
+          const float mt = fmax_(fmax_(red[st], red[64 + st]), fmax_(red[128 + st], red[192 + st]));
+          const float mu = m_use[st];
+          float al = 1.f;
+          if (mt > -INFINITY && (mu == -INFINITY || mt > mu + kLazyRescale)) {
+            al = fast_exp2(mu - mt);  // 0 when mu = -inf
+            m_use[st] = mt;
+            mine = (t > 0) && (al != 1.f);
+          }
+          alpha_s[st] = al;
+        }
+        resc = bar_red_or_128(mine);  // also the barrier that publishes m_use / alpha
+      }
 
       // the single P buffer and O are free once the previous value product is done
       if (t > 0 && !(ok = mbar_wait(p_free, uint32_t((t - 1) & 1), lim, abort_flag))) break;
@@ -424,34 +443,51 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             tmem_st16(a + 16, o + 16);
           }
         tmem_wait_st();
+#pragma unroll
+        for (int h = 0; h < 64; ++h) l_acc[h] *= alpha_s[h];
       }
-      // probabilities (bf16 for the MMA) and their per-head sums
-      float p[64];
+      // probabilities (bf16 for the MMA); the sums take the same rounded values.
+      // S is read from TMEM again, 32 heads at a time: this tile's buffer is
+      // not overwritten before P is published (the next QK into it is issued
+      // after this tile's value product).
       uint8_t* prow = smem + kPOff + r * 128;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        uint32_t w4[4];
+      for (int half = 0; half < 2; ++half) {
+        float y[32];
+        tmem_ld32_sync(lane_addr + kSCol + 64 * (t & 1) + 32 * half, y);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int h = g * 8 + 2 * u;
-          const float m0 = m_use[h], m1 = m_use[h + 1];
-          const float e0 = (valid && m0 > -INFINITY) ? fast_exp2(x[h] - m0) : 0.f;
-          const float e1 = (valid && m1 > -INFINITY) ? fast_exp2(x[h + 1] - m1) : 0.f;
-          w4[u] = pack_bf16x2(e0, e1, p[h], p[h + 1]);
+        for (int g = 0; g < 4; ++g) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int hl = g * 8 + 2 * u, h = 32 * half + hl;
+            const float m0 = m_use[h], m1 = m_use[h + 1];
+            const float e0 = (valid && m0 > -INFINITY) ? fast_exp2(y[hl] * scale_log2 - m0) : 0.f;
+            const float e1 = (valid && m1 > -INFINITY) ? fast_exp2(y[hl + 1] * scale_log2 - m1) : 0.f;
+            float q0, q1;
+            w4[u] = pack_bf16x2(e0, e1, q0, q1);
+            l_acc[h] += q0;
+            l_acc[h + 1] += q1;
+          }
+          const int gg = 4 * half + g;
+          *reinterpret_cast<uint4*>(prow + ((gg ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        *reinterpret_cast<uint4*>(prow + ((g ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
-      reduce_scatter64<false>(p, r0, r1);
-      red[rw * 64 + 2 * lane] = r0;
-      red[rw * 64 + 2 * lane + 1] = r1;
-      named_bar_sync(1, 128);
-      if (st < 64) l_run[st] += red[st] + red[64 + st] + red[128 + st] + red[192 + st];
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
     }
     // the last value product must be complete before O is read
     if (ok && ntiles > 0) mbar_wait(p_free, uint32_t((ntiles - 1) & 1), lim, abort_flag);
+    // running sums: one reduction over the tile rows
+    if (ok) {
+      float r0, r1;
+      reduce_scatter64<false>(l_acc, r0, r1);
+      red[rw * 64 + 2 * lane] = r0;
+      red[rw * 64 + 2 * lane + 1] = r1;
+      named_bar_sync(1, 128);
+      if (st < 64) l_run[st] = red[st] + red[64 + st] + red[128 + st] + red[192 + st];
+    }
   }
   // All threads: publishes l_run / m_use and makes the abort decision uniform.
   __syncthreads();

@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
       // accept x > Kf, or x == Kf at a position below P (P == INT_MAX: x >= Kf)
       float Kf = key_float(sample_threshold(row, n, topk, sh));
       int P = INT_MAX;
-      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+      const int warp = threadIdx.x >> 5;
       // Each warp appends to its own region of the buffer; [0, kept0) holds
       // the entries kept by the last cut.
       int kept0 = 0;
