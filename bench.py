@@ -207,11 +207,12 @@ def forward_streams(T: int, max_n: int) -> bool:
 
 def launches_per_step(T: int, k: int, streams: bool, sms: int) -> int:
     """Kernels of this library one dsa_forward launches: indexer plan, indexer,
-    top-k (materialised path), attention, and the split merge when rows are
+    top-k (materialised path) or the redo plan, the redo sweep and the buffer
+    selection (streamed path), attention, and the split merge when rows are
     split over several CTAs."""
     ntiles = (k + 127) // 128
     splits = max(1, min(16, ntiles, sms // max(T, 1)))
-    return 2 + (0 if streams else 1) + 1 + (1 if splits > 1 else 0)
+    return 2 + (3 if streams else 1) + 1 + (1 if splits > 1 else 0)
 
 
 def rank_seed(cfg: int, rank: int) -> int:

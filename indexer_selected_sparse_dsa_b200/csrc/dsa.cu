@@ -153,9 +153,31 @@ bool forward_streams(int T, int64_t max_n_vis) {
 }
 
 size_t ws_candidates(int T) { return align_up(size_t(T) * dsa::kStreamCap * 4, 256); }
+// streamed selection: candidate keys, candidate positions, the redo list, the candidate counts
+size_t ws_redo(int T) { return align_up((size_t(T) + 1) * 4, 256); }
+size_t ws_select(int T) { return 2 * ws_candidates(T) + ws_redo(T) + align_up(size_t(T) * 4, 256); }
+
+dsa::StreamOut stream_out_at(uint8_t* sel, int T, int32_t* idx, int topk) {
+  dsa::StreamOut so{};
+  so.cand_key = reinterpret_cast<uint32_t*>(sel);
+  so.cand_pos = reinterpret_cast<int32_t*>(sel + ws_candidates(T));
+  so.idx = idx;
+  so.topk = topk;
+  so.cap = dsa::kStreamCap;
+  so.redo = reinterpret_cast<int*>(sel + 2 * ws_candidates(T));
+  so.cnt_out = reinterpret_cast<int*>(sel + 2 * ws_candidates(T) + ws_redo(T));
+  so.sample_units = dsa::kSampleUnits;
+  so.sample_mode = 1;
+  // DSA_STREAM_SAMPLE=0: no seeding; =2: seed at the sample maximum (tests of the redo sweep)
+  if (const char* m = std::getenv("DSA_STREAM_SAMPLE")) {
+    if (m[0] == '0') so.sample_units = 0;
+    if (m[0] == '2') so.sample_mode = 2;
+  }
+  return so;
+}
 
 size_t ws_forward(int T, int64_t max_n_vis, int topk) {
-  const size_t sel = forward_streams(T, max_n_vis) ? 2 * ws_candidates(T)
+  const size_t sel = forward_streams(T, max_n_vis) ? ws_select(T)
                                                    : align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256);
   return ws_indexer(T) + sel + align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
 }
@@ -227,6 +249,8 @@ int run_indexer(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int
   p.stream = stream;
   cudaError_t e = dsa::launch_indexer(p, tk, tq);
   if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+  if (stream_out && (e = dsa::launch_stream_select(*stream_out, n_vis, T, stream)) != cudaSuccess)
+    return cuda_fail(e, "streamed top-k launch");
   return DSA_OK;
 }
 
@@ -247,7 +271,7 @@ size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
     case DSA_OP_TOPK: return 0;
     case DSA_OP_SPARSE_MLA: return ws_mla(T, topk);
     case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
-    case DSA_OP_INDEXER_TOPK: return ws_indexer(T) + 2 * ws_candidates(T);
+    case DSA_OP_INDEXER_TOPK: return ws_indexer(T) + ws_select(T);
     default: return 0;
   }
 }
@@ -328,7 +352,7 @@ int dsa_indexer_topk(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I
     return fail(DSA_ERR_INVALID_ARG, "q_I, w, k_I must be 16-byte aligned; n_vis, idx 4-byte aligned");
   if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
   if (int64_t(T) * DSA_INDEX_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
-  const size_t need = ws_indexer(T) + 2 * ws_candidates(T);
+  const size_t need = ws_indexer(T) + ws_select(T);
   if (ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, need);
   DeviceState* dev = nullptr;
   if ((rc = current_device(&dev))) return rc;
@@ -336,8 +360,7 @@ int dsa_indexer_topk(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I
   uint8_t* sel = base + ws_indexer(T);
   cudaError_t e = cudaMemsetAsync(idx, 0xFF, size_t(T) * size_t(topk) * 4, stream);  // rejected rows stay -1
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(idx)");
-  dsa::StreamOut so{reinterpret_cast<uint32_t*>(sel), reinterpret_cast<int32_t*>(sel + ws_candidates(T)), idx, topk,
-                    dsa::kStreamCap};
+  const dsa::StreamOut so = stream_out_at(sel, T, idx, topk);
   return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, nullptr, score_ld_for(max_n_vis), base, stream,
                      dev->sm_count, &so);
 }
@@ -370,7 +393,7 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   uint8_t* base = static_cast<uint8_t*>(ws);
   void* plan = base;
   uint8_t* sel = base + ws_indexer(T);  // score matrix, or the candidate buffers
-  const size_t sel_bytes = streams ? 2 * ws_candidates(T) : align_up(size_t(T) * size_t(ld) * 4, 256);
+  const size_t sel_bytes = streams ? ws_select(T) : align_up(size_t(T) * size_t(ld) * 4, 256);
   int32_t* idx_ws = reinterpret_cast<int32_t*>(sel + sel_bytes);
   int32_t* idx = idx_out ? idx_out : idx_ws;
   float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(idx_ws) + align_up(size_t(T) * size_t(topk) * 4, 256));
@@ -380,8 +403,7 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
     // Rows the indexer plan rejects are never visited: they keep -1 everywhere.
     if ((e = cudaMemsetAsync(idx, 0xFF, size_t(T) * size_t(topk) * 4, stream)) != cudaSuccess)
       return cuda_fail(e, "cudaMemsetAsync(idx)");
-    dsa::StreamOut so{reinterpret_cast<uint32_t*>(sel), reinterpret_cast<int32_t*>(sel + ws_candidates(T)), idx,
-                      topk, dsa::kStreamCap};
+    const dsa::StreamOut so = stream_out_at(sel, T, idx, topk);
     if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, nullptr, ld, plan, stream, dev->sm_count,
                           &so)))
       return rc;

@@ -1,7 +1,7 @@
 // Selection helpers for a group of warps inside a warp-specialised CTA (the
-// indexer's epilogue warps): scans, exact radix select, in-place compaction
-// and a bitonic sort, synchronised with one named barrier instead of
-// __syncthreads so the other roles of the CTA keep running.
+// indexer's epilogue warps): scans, exact radix select and in-place
+// compaction, synchronised with one named barrier instead of __syncthreads so
+// the other roles of the CTA keep running.
 #pragma once
 #include <cstdint>
 
@@ -10,6 +10,8 @@
 namespace dsa {
 
 namespace {
+
+constexpr int kBatch = 8;  // entries per thread in flight in the selection loops
 
 struct Group {
   int tid;  // 0 .. n-1
@@ -61,6 +63,7 @@ __device__ __forceinline__ int group_exclusive_sum(int v, GroupShared& gs, int* 
 struct Rule {
   long long thr;  // keep key > thr ...
   int keep_eq;    // ... and the first keep_eq keys == thr (by the caller's tie order)
+  int count_eq;   // how many entries have key == thr (when keep_eq > 0)
 };
 
 // Exact selection of the need-th largest key among the m entries with inc(j);
@@ -77,10 +80,20 @@ __device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared&
     const int nb = 1 << w;
     for (int b = g.tid; b < nb; b += g.n) hist[b] = 0u;
     g.sync();
-    for (int j = g.tid; j < m; j += g.n) {
-      if (!inc(j)) continue;
-      const uint32_t k = key(j);
-      if (bits_done == 0 || (k >> (32 - bits_done)) == prefix) atomicAdd(&hist[(k >> shift) & uint32_t(nb - 1)], 1u);
+    // entries may sit in global memory: kBatch loads in flight per thread
+    for (int j0 = g.tid; j0 < m; j0 += g.n * kBatch) {
+      uint32_t kk[kBatch];
+      bool in[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = j0 + u * g.n;
+        in[u] = j < m && inc(j);
+        kk[u] = in[u] ? key(j) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (in[u] && (bits_done == 0 || (kk[u] >> (32 - bits_done)) == prefix))
+          atomicAdd(&hist[(kk[u] >> shift) & uint32_t(nb - 1)], 1u);
     }
     g.sync();
     // bin where the count from the top first reaches `need`
@@ -109,51 +122,41 @@ __device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared&
     prefix = (prefix << w) | uint32_t(gs.sel_bin);
     need -= gs.sel_above;
     bits_done += w;
-    const bool whole = (gs.sel_count == need);
+    const int count = gs.sel_count;
     g.sync();
-    if (whole) return Rule{((long long)prefix << (32 - bits_done)) - 1, 0};
+    if (count == need) return Rule{((long long)prefix << (32 - bits_done)) - 1, 0, 0};
+    if (p == 2) return Rule{(long long)prefix, need, count};
   }
-  return Rule{(long long)prefix, need};
+  return Rule{0, 0, 0};  // not reached
 }
 
 // In-place stable compaction: entry j (read with load(j)) is kept when keep(e);
-// kept entries are written to the front with store(dst, e), dst <= j.  Every
-// entry of a chunk is loaded into registers before any store of that chunk
-// (the scan's barriers separate them).  Returns how many were kept.
+// kept entries are written to the front with store(dst, e), dst <= j.  Each
+// round covers kBatch consecutive entries per thread, all loaded into registers
+// before any store of the round (the scan's barriers separate them).  Returns
+// how many were kept.
 template <class Load, class Keep, class Store>
 __device__ int group_compact(int m, GroupShared& gs, const Group& g, Load load, Keep keep, Store store) {
   int written = 0;
-  for (int base = 0; base < m; base += g.n) {
-    const int j = base + g.tid;
-    auto e = load(j < m ? j : 0);
-    const bool k = j < m && keep(e);
+  for (int base = 0; base < m; base += g.n * kBatch) {
+    const int j0 = base + g.tid * kBatch;
+    decltype(load(0)) e[kBatch];
+    unsigned km = 0u;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (j0 + u < m) {
+        e[u] = load(j0 + u);
+        if (keep(e[u])) km |= 1u << u;
+      }
     int tot = 0;
-    const int o = written + group_exclusive_sum(k ? 1 : 0, gs, &tot, g);
-    if (k) store(o, e);
+    int o = written + group_exclusive_sum(__popc(km), gs, &tot, g);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if ((km >> u) & 1u) store(o++, e[u]);
     g.sync();
     written += tot;
   }
   return written;
-}
-
-// Ascending bitonic sort of buf[0, npow2) (npow2 a power of two).
-__device__ void group_bitonic_sort(int* buf, int npow2, const Group& g) {
-  for (int k = 2; k <= npow2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = g.tid; i < npow2; i += g.n) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const bool asc = (i & k) == 0;
-          const int a = buf[i], b = buf[ixj];
-          if ((a > b) == asc) {
-            buf[i] = b;
-            buf[ixj] = a;
-          }
-        }
-      }
-      g.sync();
-    }
-  }
 }
 
 }  // namespace

@@ -18,10 +18,20 @@
 // Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
 // and MMA issuer, warps 2..9 = epilogue (two warps per TMEM lane quarter, each
 // taking every other query of the tile).  Persistent grid.
+//
+// Streamed selection (STREAM): no score is written.  Each score above its
+// query's filter threshold goes, with its position, into the query's
+// candidate buffer (workspace, kStreamCap entries).  A long tile first scores
+// kSampleUnits key units spread over its range and seeds every threshold from
+// them; every kCheckUnits units a buffer that could overflow is cut to its
+// exact top-k and its threshold raised to the k-th score.  The exact top-k of
+// the final buffers is taken afterwards by launch_stream_select; rows whose
+// seeded filter let too few keys through are swept again unseeded first.
 #pragma once
 #include <cuda.h>
 
 #include "block_scan.cuh"
+#include "dsa.h"
 #include "group_select.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -128,15 +138,52 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(const int64_t* __res
   }
 }
 
+// Plan of the redo sweep: one tile per query listed in redo[1 .. redo[0]].
+__global__ void __launch_bounds__(1024) indexer_redo_plan_kernel(const int* __restrict__ redo,
+                                                                 const int64_t* __restrict__ kv_start,
+                                                                 const int32_t* __restrict__ n_vis,
+                                                                 PlanHeader* __restrict__ hdr,
+                                                                 PlanTile* __restrict__ tiles) {
+  __shared__ long long sc_l[33];
+  const int n = redo[0];
+  long long carry = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int j = base + threadIdx.x;
+    long long u = 0;
+    PlanTile t{};
+    if (j < n) {
+      const int q = redo[1 + j];
+      t.q0 = q;
+      t.nq = 1;
+      t.units = (n_vis[q] + kKeysPerUnit - 1) / kKeysPerUnit;
+      t.kv_start = kv_start[q];
+      u = t.units;
+    }
+    long long total = 0;
+    const long long ex = block_exclusive_sum<long long>(u, sc_l, &total);
+    if (j < n) {
+      t.unit_begin = carry + ex;
+      tiles[j] = t;
+    }
+    carry += total;
+  }
+  if (threadIdx.x == 0) {
+    hdr->total_units = carry;
+    hdr->n_tiles = n;
+  }
+}
+
 // ------------------------------------------------------------------ unit iterator
 // Every role of the main kernel walks the same sequence of (query tile, key tile).
 struct UnitIter {
   const PlanTile* tiles;
   int n_tiles;
   int sweep;
+  int samples = 0;  // sample units ahead of a long tile's sweep (wave sweep only)
   int tile;
-  int kt;
-  long long left;  // units left (split sweep)
+  int kt;           // step within the tile: -ns .. -1 sample units, then 0 .. units-1
+  int ns;           // this tile's sample units
+  long long left;   // units left (split sweep)
   PlanTile cur;
 
   __device__ bool load_tile(int j) {
@@ -144,16 +191,22 @@ struct UnitIter {
     if (j >= n_tiles) return false;
     tile = j;
     cur = tiles[j];
+    ns = (samples > 0 && cur.units >= kSampleMinUnits) ? samples : 0;
     return true;
   }
+  // key unit of the current step; sample unit i of ns is unit i * units / ns
+  __device__ int unit() const { return kt >= 0 ? kt : int((long long)(kt + ns) * cur.units / ns); }
   __device__ bool begin(const PlanHeader* hdr, const PlanTile* t) {
     tiles = t;
     n_tiles = hdr->n_tiles;
     const long long U = hdr->total_units;
     kt = 0;
+    ns = 0;
     if (sweep == kSweepWave) {
       left = 1;
-      return load_tile(int(blockIdx.x));
+      if (!load_tile(int(blockIdx.x))) return false;
+      kt = -ns;
+      return true;
     }
     const long long G = gridDim.x;
     const long long b = U * (long long)blockIdx.x / G, e = U * (long long)(blockIdx.x + 1) / G;
@@ -176,15 +229,18 @@ struct UnitIter {
       if (--left <= 0) return false;
     }
     if (kt < cur.units) return true;
-    kt = 0;
-    return load_tile(tile + (sweep == kSweepWave ? int(gridDim.x) : 1));
+    if (!load_tile(tile + (sweep == kSweepWave ? int(gridDim.x) : 1))) return false;
+    kt = -ns;
+    return true;
   }
 };
 
 // ------------------------------------------------------------------ main kernel
 constexpr int kEpiWarps = 8;
 constexpr int kIdxThreads = 64 + 32 * kEpiWarps;
-constexpr int kCheckUnits = 8;  // streaming selection: units between candidate-buffer checks
+constexpr int kCheckUnits = 32;  // streaming selection: units between candidate-buffer checks
+static_assert(kStreamCap - DSA_MAX_TOPK >= kCheckUnits * kKeysPerUnit,
+              "a cut buffer must take every key of one check interval");
 
 template <int QMAX, int STAGES, int QBUF, bool STREAM>
 struct IdxSmem {
@@ -196,10 +252,10 @@ struct IdxSmem {
   // streaming selection state: thresholds, counts, scan scratch, histogram, sort buffer
   static constexpr int kThrOff = (kNvOff + QMAX * 4 + 15) & ~15;      // long long thr[QMAX]
   static constexpr int kCntOff = kThrOff + QMAX * 8;                  // int cnt[QMAX]
-  static constexpr int kGsOff = kCntOff + QMAX * 4;                   // GroupShared
+  static constexpr int kSmpOff = kCntOff + QMAX * 4;                  // int seeded[QMAX]
+  static constexpr int kGsOff = kSmpOff + QMAX * 4;                   // GroupShared
   static constexpr int kHistOff = (kGsOff + int(sizeof(GroupShared)) + 15) & ~15;  // uint32 hist[4096]
-  static constexpr int kSortOff = kHistOff + 4096 * 4;                // int sort[2048]
-  static constexpr int kStreamEnd = STREAM ? kSortOff + 2048 * 4 : kNvOff + QMAX * 4;
+  static constexpr int kStreamEnd = STREAM ? kHistOff + 4096 * 4 : kNvOff + QMAX * 4;
   static constexpr int kBarOff = (kStreamEnd + 7) & ~7;
   static constexpr int kNumBars = 2 * STAGES + 2 * QBUF + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;             // tmem slot, abort flag
@@ -267,6 +323,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (lane == 0) {
       UnitIter it;
       it.sweep = sweep;
+      it.samples = STREAM ? so.sample_units : 0;
       int stage = 0, qb = -1, prev_tile = -1;
       uint32_t phase = 0;
       uint32_t qphase[QBUF];
@@ -291,7 +348,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, lim, abort_flag)) break;
         mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
-        const int y = int(it.cur.kv_start + (long long)it.kt * kKeysPerUnit);
+        const int y = int(it.cur.kv_start + (long long)it.unit() * kKeysPerUnit);
         const uint32_t kdst = sbase + L::kKeysOff + stage * kStageBytes;
         tma_load_2d(kdst, &tmap_k, full_bar(stage), 0, y);
         tma_load_2d(kdst + kHalfKeyBytes, &tmap_k, full_bar(stage), 64, y);
@@ -311,6 +368,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (lane == 0) {
       UnitIter it;
       it.sweep = sweep;
+      it.samples = STREAM ? so.sample_units : 0;
       int stage = 0, qb = -1, prev_tile = -1, ab = 0;
       uint32_t phase = 0, aphase = 0;
       uint32_t qphase[QBUF];
@@ -363,9 +421,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int et = threadIdx.x - 64;      // 0 .. 32 * kEpiWarps - 1
     long long* thr_s = reinterpret_cast<long long*>(smem + L::kThrOff);
     int* cnt_s = reinterpret_cast<int*>(smem + L::kCntOff);
+    int* seeded_s = reinterpret_cast<int*>(smem + L::kSmpOff);
     GroupShared& gs = *reinterpret_cast<GroupShared*>(smem + L::kGsOff);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L::kHistOff);
-    int* sortbuf = reinterpret_cast<int*>(smem + L::kSortOff);
     // Keep the topk best entries of query q's buffer (exact: ties at the cut go to the
     // lowest positions), move them to its front and raise its filter threshold.
     auto stream_shrink = [&](int q, int q0, const Group& g) {
@@ -377,7 +435,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const Rule r = group_radix_select(m, so.topk, hist, gs, g, [&](int j) { return ck[j]; },
                                         [](int) { return true; });
       long long cut = 0;  // among keys == r.thr keep positions p with ~p >= cut
-      if (r.keep_eq > 0) {
+      if (r.keep_eq > 0 && r.keep_eq < r.count_eq) {  // some tied keys must go: lowest positions stay
         const Rule rp = group_radix_select(
             m, r.keep_eq, hist, gs, g, [&](int j) { return ~uint32_t(cp[j]); },
             [&](int j) { return (long long)ck[j] == r.thr; });
@@ -399,22 +457,62 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
       g.sync();
     };
-    // Final selection of query q: its kept positions, ascending, padded with -1.
-    auto stream_finish = [&](int q, int q0, const Group& g) {
-      stream_shrink(q, q0, g);
+    // After the sample units: start query q's filter at a threshold that about
+    // (1 + 4 / sqrt(share)) x topk of its keys should pass, share being the
+    // sample's expected part of its topk; the buffer is emptied (the main sweep
+    // visits the sampled keys again).  Rows that fit the buffer keep every key.
+    auto stream_seed = [&](int q, int q0, const Group& g) {
       const long long ro = (long long)(q0 + q) * so.cap;
-      const int m = min(cnt_s[q], so.topk);
-      int np2 = 1;
-      while (np2 < m) np2 <<= 1;
-      for (int j = g.tid; j < np2; j += g.n) sortbuf[j] = j < m ? so.cand_pos[ro + j] : 0x7fffffff;
+      const int S = min(cnt_s[q], so.cap);
+      const int n = nv_s[q];
+      long long t = -1;
+      int seeded = 0;
+      if (n > so.cap && S > 0) {
+        int r = 1;
+        if (so.sample_mode != 2) {
+          const float share = float(so.topk) * float(S) / float(n);
+          r = int(ceilf(share + 4.0f * sqrtf(share))) + 8;
+        }
+        if (r < S) {
+          const Rule rr = group_radix_select(S, r, hist, gs, g, [&](int j) { return so.cand_key[ro + j]; },
+                                             [](int) { return true; });
+          t = rr.keep_eq > 0 ? rr.thr - 1 : rr.thr;  // keys >= the r-th largest sample key pass
+          seeded = 1;
+        }
+      }
+      if (g.tid == 0) {
+        thr_s[q] = t;
+        cnt_s[q] = 0;
+        seeded_s[q] = seeded;
+      }
       g.sync();
-      group_bitonic_sort(sortbuf, np2, g);
-      int32_t* out = so.idx + (long long)(q0 + q) * so.topk;
-      for (int j = g.tid; j < so.topk; j += g.n) out[j] = j < m ? sortbuf[j] : -1;
-      g.sync();
+    };
+    // End of query q's sweep: hand its candidate count to the selection kernel
+    // that runs after the sweeps (exact top-k of the buffer, written ascending).
+    // A seeded filter that let fewer than min(topk, n) keys through (no cut
+    // happened, or cnt would be >= topk) may have dropped some of the best: the
+    // query goes on the redo list instead and is swept again unseeded.
+    auto stream_finish = [&](int q, int q0) {
+      if (et != 0) return;
+      if (seeded_s[q] && cnt_s[q] < min(so.topk, nv_s[q])) so.redo[1 + atomicAdd(so.redo, 1)] = q0 + q;
+      else so.cnt_out[q0 + q] = min(cnt_s[q], so.cap);
+    };
+    // This thread's queries are half, half + 2, half + 4, half + 6 (slot j: half + 2j);
+    // their visible lengths and filter thresholds live in registers, reloaded from
+    // shared memory only where they change (tile start, seeding, buffer checks).
+    int nv_r[4];
+    long long thr_r[4];
+    auto refresh = [&]() {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = half + 2 * j;
+        nv_r[j] = q < QMAX ? nv_s[q] : 0;
+        thr_r[j] = (STREAM && q < QMAX) ? thr_s[q] : -1;
+      }
     };
     UnitIter it;
     it.sweep = sweep;
+    it.samples = STREAM ? so.sample_units : 0;
     int prev_tile = -1, ab = 0;
     uint32_t aphase = 0;
     bool ok = it.begin(hdr, tiles);
@@ -424,91 +522,127 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         named_bar_sync(1, 32 * kEpiWarps);
         for (int e = et; e < nq * 32; e += 32 * kEpiWarps)
           w_s[e] = bf16_bits_to_float(w[(long long)it.cur.q0 * 32 + e]);
-        if (et < nq) nv_s[et] = n_vis[it.cur.q0 + et];
+        if (et < QMAX) nv_s[et] = et < nq ? n_vis[it.cur.q0 + et] : 0;
         if constexpr (STREAM) {
           if (et < QMAX) {
             thr_s[et] = -1;  // nothing kept yet: every score passes
             cnt_s[et] = 0;
+            seeded_s[et] = 0;
           }
         }
         named_bar_sync(1, 32 * kEpiWarps);
+        refresh();
         prev_tile = it.tile;
       }
       if (!mbar_wait(afull_bar(ab), aphase, lim, abort_flag)) break;
       tc_fence_after();
-      const long long s = (long long)it.kt * kKeysPerUnit + row;
+      const long long s = (long long)it.unit() * kKeysPerUnit + row;
       const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
       // score of (query qi, key s): written out, or offered to the query's candidate buffer
-      auto emit = [&](int qi, float score) {
-        const bool in = s < nv_s[qi];
-        if constexpr (!STREAM) {
-          if (in) scores[(long long)(it.cur.q0 + qi) * score_ld + s] = score;
-        } else {
-          const uint32_t key = float_order_key(score);
-          const bool pass = in && (long long)key > thr_s[qi];
-          const unsigned m = __ballot_sync(0xffffffffu, pass);
-          if (m) {
-            const int leader = __ffs(m) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&cnt_s[qi], __popc(m));
-            base = __shfl_sync(0xffffffffu, base, leader);
-            const int off = base + __popc(m & ((1u << lane) - 1u));
-            if (pass && off < so.cap) {
-              const long long ro = (long long)(it.cur.q0 + qi) * so.cap;
-              so.cand_key[ro + off] = key;
-              so.cand_pos[ro + off] = int(s);
-            }
+      // append the passing scores of query slot j (qi = half + 2j) to its buffer
+      auto append = [&](int j, uint32_t key, bool pass) {
+        const int qi = half + 2 * j;
+        const unsigned m = __ballot_sync(0xffffffffu, pass);
+        if (m) {
+          const int leader = __ffs(m) - 1;
+          int base = 0;
+          if (lane == leader) base = atomicAdd(&cnt_s[qi], __popc(m));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          const int off = base + __popc(m & ((1u << lane) - 1u));
+          if (pass && off < so.cap) {
+            const long long ro = (long long)(it.cur.q0 + qi) * so.cap;
+            so.cand_key[ro + off] = key;
+            so.cand_pos[ro + off] = int(s);
           }
         }
       };
-      // this warp's queries, two per TMEM wait: qi = half, half + 2 (then + 4, + 6)
-      for (int qi = half; qi < nq; qi += 4) {
-        const int qj = qi + 2;
-        float v[64];
-        if (qj < nq) {
-          tmem_ld32x2_sync(tbase + uint32_t(qi * 32), tbase + uint32_t(qj * 32), v);
-        } else {
-          tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
-        }
-        const float4* w0 = reinterpret_cast<const float4*>(w_s + qi * 32);
-        float a0 = 0.f, a1 = 0.f;
+      // This warp's queries, two per TMEM wait: qi = half, half + 2 (then + 4, + 6).
+      // All scores are computed first and the accumulator is handed back to the
+      // MMA warp before any is written or offered to a selection buffer.
+      float sc[4];
 #pragma unroll
-        for (int h4 = 0; h4 < 8; ++h4) {
-          const float4 c = w0[h4];
-          a0 = fmaf(c.x, v[4 * h4], a0);
-          a0 = fmaf(c.y, v[4 * h4 + 1], a0);
-          a0 = fmaf(c.z, v[4 * h4 + 2], a0);
-          a0 = fmaf(c.w, v[4 * h4 + 3], a0);
-        }
-        emit(qi, a0);
-        if (qj < nq) {
-          const float4* w1 = reinterpret_cast<const float4*>(w_s + qj * 32);
+      for (int it2 = 0; it2 < 2; ++it2) {
+        const int qi = half + 4 * it2, qj = qi + 2;
+        sc[2 * it2] = sc[2 * it2 + 1] = 0.f;
+        if (qi < nq) {
+          float v[64];
+          if (qj < nq) {
+            tmem_ld32x2_sync(tbase + uint32_t(qi * 32), tbase + uint32_t(qj * 32), v);
+          } else {
+            tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
+          }
+          const float4* w0 = reinterpret_cast<const float4*>(w_s + qi * 32);
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 c = w1[h4];
-            a1 = fmaf(c.x, v[32 + 4 * h4], a1);
-            a1 = fmaf(c.y, v[32 + 4 * h4 + 1], a1);
-            a1 = fmaf(c.z, v[32 + 4 * h4 + 2], a1);
-            a1 = fmaf(c.w, v[32 + 4 * h4 + 3], a1);
+            const float4 c = w0[h4];
+            a0 = fmaf(c.x, v[4 * h4], a0);
+            a0 = fmaf(c.y, v[4 * h4 + 1], a0);
+            a0 = fmaf(c.z, v[4 * h4 + 2], a0);
+            a0 = fmaf(c.w, v[4 * h4 + 3], a0);
           }
-          emit(qj, a1);
+          if (qj < nq) {
+            const float4* w1 = reinterpret_cast<const float4*>(w_s + qj * 32);
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              const float4 c = w1[h4];
+              a1 = fmaf(c.x, v[32 + 4 * h4], a1);
+              a1 = fmaf(c.y, v[32 + 4 * h4 + 1], a1);
+              a1 = fmaf(c.z, v[32 + 4 * h4 + 2], a1);
+              a1 = fmaf(c.w, v[32 + 4 * h4 + 3], a1);
+            }
+          }
+          sc[2 * it2] = a0;
+          sc[2 * it2 + 1] = a1;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(aempty_bar(ab));
+      if constexpr (!STREAM) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (s < nv_r[j]) scores[(long long)(it.cur.q0 + half + 2 * j) * score_ld + s] = sc[j];
+      } else {
+        // one vote for the common case that no score of the warp passes its filter
+        uint32_t key[4];
+        bool pass[4];
+        bool any = false;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          key[j] = float_order_key(sc[j]);
+          pass[j] = s < nv_r[j] && (long long)key[j] > thr_r[j];
+          any = any || pass[j];
+        }
+        if (__any_sync(0xffffffffu, any)) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (half + 2 * j < nq) append(j, key[j], pass[j]);
+        }
+      }
       if constexpr (STREAM) {
-        // Every kCheckUnits units: shrink buffers that could overflow before the next
-        // check (a query gains at most one entry per key); after the tile's last unit,
-        // finish its queries.
-        const bool last = it.kt == it.cur.units - 1;
-        if (last || (it.kt % kCheckUnits) == kCheckUnits - 1) {
-          const Group g{et, 32 * kEpiWarps, 1};
-          g.sync();
-          for (int q = 0; q < nq; ++q)
-            if (cnt_s[q] > so.cap - kCheckUnits * kKeysPerUnit) stream_shrink(q, it.cur.q0, g);
-          if (last)
-            for (int q = 0; q < nq; ++q) stream_finish(q, it.cur.q0, g);
+        const Group g{et, 32 * kEpiWarps, 1};
+        if (it.kt < 0) {
+          // the sample units fill at most kSampleUnits * 128 = cap entries; after
+          // the last one, seed each query's threshold
+          if (it.kt == -1) {
+            g.sync();
+            for (int q = 0; q < nq; ++q) stream_seed(q, it.cur.q0, g);
+            refresh();
+          }
+        } else {
+          // Every kCheckUnits units: shrink buffers that could overflow before the
+          // next check (a query gains at most one entry per key); after the tile's
+          // last unit, finish its queries.
+          const bool last = it.kt == it.cur.units - 1;
+          if (last || (it.kt % kCheckUnits) == kCheckUnits - 1) {
+            g.sync();
+            for (int q = 0; q < nq; ++q)
+              if (cnt_s[q] > so.cap - kCheckUnits * kKeysPerUnit) stream_shrink(q, it.cur.q0, g);
+            if (last)
+              for (int q = 0; q < nq; ++q) stream_finish(q, it.cur.q0);
+            refresh();
+          }
         }
       }
       if (++ab == 2) {
@@ -559,13 +693,29 @@ cudaError_t prepare_indexer() {
 
 cudaError_t launch_indexer(const IndexerLaunch& p, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q) {
   if (p.T <= 0) return cudaSuccess;
+  static_assert(kSampleUnits * kKeysPerUnit <= kStreamCap, "the sample fills at most the candidate buffer");
+  if (p.streaming) {
+    cudaError_t e0 = cudaMemsetAsync(p.stream_out.redo, 0, sizeof(int), p.stream);
+    if (e0 == cudaSuccess) e0 = cudaMemsetAsync(p.stream_out.cnt_out, 0xFF, size_t(p.T) * 4, p.stream);
+    if (e0 != cudaSuccess) return e0;
+  }
   auto* hdr = reinterpret_cast<PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<PlanTile*>(reinterpret_cast<uint8_t*>(p.plan) + sizeof(PlanHeader));
   indexer_plan_kernel<<<1, 1024, 0, p.stream>>>(p.kv_start, p.n_vis, p.T, p.qmax, p.score_ld, p.cache_rows, hdr,
                                                 tiles);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (p.streaming) return p.qmax == 8 ? launch_main<8, 4, 1, true>(p, tmap_k, tmap_q) : cudaErrorInvalidValue;
+  if (p.streaming) {
+    if (p.qmax != 8 || p.sweep != kSweepWave) return cudaErrorInvalidValue;
+    if ((e = launch_main<8, 4, 1, true>(p, tmap_k, tmap_q)) != cudaSuccess) return e;
+    // queries whose seeded threshold let too few keys through: sweep them again,
+    // unseeded (an empty list costs one short launch, no host round trip)
+    indexer_redo_plan_kernel<<<1, 1024, 0, p.stream>>>(p.stream_out.redo, p.kv_start, p.n_vis, hdr, tiles);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    IndexerLaunch p2 = p;
+    p2.stream_out.sample_units = 0;
+    return launch_main<8, 4, 1, true>(p2, tmap_k, tmap_q);
+  }
   switch (p.qmax) {
     case 1: return launch_main<1, 6, 2, false>(p, tmap_k, tmap_q);
     case 4: return launch_main<4, 4, 2, false>(p, tmap_k, tmap_q);

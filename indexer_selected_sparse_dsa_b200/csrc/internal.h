@@ -43,8 +43,20 @@ struct StreamOut {
   int32_t* idx;        // [T, topk]
   int topk;
   int cap;
+  // Threshold seeding: before its sweep, a long query tile scores sample_units
+  // key units spread over its range and starts each query's filter at a
+  // threshold that about (1 + 4 / sqrt(share)) x topk of its keys pass
+  // (sample_mode 2: at the sample's maximum, which lets too few pass; a test
+  // of the redo pass).  A query with fewer than topk passing keys at the end
+  // is listed in redo[1 + i] (redo[0] counts them) and swept again unseeded.
+  int* redo;           // [1 + T]
+  int* cnt_out;        // [T]: candidates left in a query's buffer after its sweep (-1: none yet)
+  int sample_units;
+  int sample_mode;
 };
 constexpr int kStreamCap = 8192;
+constexpr int kSampleUnits = 64;        // 8192 keys: fits the candidate buffer
+constexpr int kSampleMinUnits = 1024;   // tiles of at least 128K keys are seeded
 
 struct IndexerLaunch {
   const uint16_t* q_I;
@@ -97,5 +109,8 @@ cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q);
 cudaError_t prepare_indexer();
 cudaError_t prepare_sparse_mla();
 cudaError_t prepare_topk();
+// Exact top-k of each query's candidate buffer (after the streamed sweep),
+// written ascending and -1 padded; rows with cnt_out < 0 are left as they are.
+cudaError_t launch_stream_select(const StreamOut& so, const int32_t* n_vis, int T, cudaStream_t stream);
 
 }  // namespace dsa

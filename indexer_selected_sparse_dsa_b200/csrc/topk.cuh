@@ -593,10 +593,47 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   }
 }
 
+// Exact top-k of the candidate buffers a streamed indexer sweep leaves (one CTA
+// per query row): the buffer's (key, position) pairs, in no particular order,
+// are loaded into shared memory, selected (ties to lower positions) and written
+// ascending through the position bitmap.  A row with cnt < 0 was never swept.
+__global__ void __launch_bounds__(kTopkThreads) stream_select_kernel(const uint32_t* __restrict__ cand_key,
+                                                                     const int32_t* __restrict__ cand_pos,
+                                                                     const int* __restrict__ cnt, int cap,
+                                                                     const int32_t* __restrict__ n_vis, int topk,
+                                                                     int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t topk_smem[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  const int r = blockIdx.x;
+  const int m = min(cnt[r], cap);
+  if (m < 0) return;
+  const long long ro = (long long)r * cap;
+  for (int j = threadIdx.x; j < m; j += kTopkThreads) {
+    sh.cand_key[j] = cand_key[ro + j];
+    sh.cand_pos[j] = cand_pos[ro + j];
+  }
+  __syncthreads();
+  Selection sel{-1, 0, -1, 0};  // fewer than topk candidates: keep them all
+  if (m > topk) sel = select_candidates(m, topk, sh);
+  write_selected(m, n_vis[r], sel, topk, idx + (long long)r * topk, sh);
+}
+
 }  // namespace
 
 cudaError_t prepare_topk() {
-  return cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(TopkShared)));
+  cudaError_t e =
+      cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(TopkShared)));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(stream_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(sizeof(TopkShared)));
+}
+
+cudaError_t launch_stream_select(const StreamOut& so, const int32_t* n_vis, int T, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  static_assert(kStreamCap <= kCandCap, "a streamed candidate buffer fits the shared candidate arrays");
+  stream_select_kernel<<<T, kTopkThreads, sizeof(TopkShared), stream>>>(so.cand_key, so.cand_pos, so.cnt_out, so.cap,
+                                                                       n_vis, so.topk, so.idx);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk, int32_t* idx,

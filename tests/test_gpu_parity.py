@@ -353,11 +353,41 @@ def test_forward_streamed_ties_go_to_lowest_positions(monkeypatch):
     assert np.array_equal(idx, idx_m)
 
 
+def _seeded_all_equal():
+    c = wl.make_case_numpy([140000], [(0, 140000), (0, 139000), (0, 131072), (0, 20000)], seed=66, n_plant=0)
+    c.k_I[:] = c.k_I[0]          # every score of a query is the same value
+    return c
+
+
+# One query tile over more than 128K keys: its filters are seeded from 64 sampled key units.
+SEEDED_CASES = {
+    "seeded_long": lambda: wl.make_case_numpy(
+        [200000], [(0, 200000), (0, 199999), (0, 180000), (0, 150000), (0, 131072), (0, 70000), (0, 9000),
+                   (0, 3000)], seed=64),
+    "seeded_two_tiles": lambda: wl.make_case_numpy(
+        [160000], [(0, 160000 - 3 * i) for i in range(11)], seed=65),
+    "seeded_all_equal": _seeded_all_equal,
+}
+
+
+@pytest.mark.parametrize("mode", ["1", "2", "0"])
+@pytest.mark.parametrize("name", sorted(SEEDED_CASES))
+def test_indexer_topk_seeded_equals_scores_then_topk(name, mode, monkeypatch):
+    """Seeded filters (mode 1), seeds at the sample maximum that send rows to the
+    redo sweep (mode 2), and no seeding (mode 0) all select exactly what
+    dsa_indexer_scores + dsa_topk select."""
+    monkeypatch.setenv("DSA_STREAM_SAMPLE", mode)
+    _check_indexer_topk(SEEDED_CASES[name]())
+
+
 @pytest.mark.parametrize("name", sorted(STREAM_CASES))
 def test_indexer_topk_equals_scores_then_topk(name):
     """The fused entry point selects exactly what dsa_indexer_scores + dsa_topk select."""
+    _check_indexer_topk(STREAM_CASES[name]())
+
+
+def _check_indexer_topk(c):
     import torch
-    c = STREAM_CASES[name]()
     d = to_dev(c)
     T, maxn, k = c.T, int(max(c.n_vis)), 2048
     ld = (maxn + 3) // 4 * 4
