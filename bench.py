@@ -1,7 +1,8 @@
 """Benchmark of the DSA sparse-attention step (indexer -> top-k -> sparse MLA).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config C] [--scale S] [--skip-cpu] [--skip-e2e]
+                    [--config C] [--scale S] [--skip-cpu] [--skip-e2e] [--indexshare L]
+                    [--dense-window W]
 
 One step = one dsa_forward over one batch of the workload (every query row:
 indexer over its causal context, exact top-2048, sparse latent MLA).  The
@@ -13,6 +14,13 @@ path has no data exchange between rows).  Rank 0 prints one JSON line.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload shape
 (rank 0 only; bounded samples of query rows per step).
+
+``--indexshare L`` times an IndexShare group instead: one step runs the full
+layer (dsa_forward) and L-1 layers that reuse its index set
+(dsa_sparse_mla_attn with their own queries and latent caches); the line
+adds the full-layer and shared-layer times.  ``--dense-window W`` times the
+dense + sparse layer: the selection, then dsa_dense_sparse_attn (attention over
+the selected set and over the last W positions, fused per head).
 """
 from __future__ import annotations
 
@@ -215,6 +223,12 @@ def launches_per_step(T: int, k: int, streams: bool, sms: int) -> int:
     return 2 + (3 if streams else 1) + 1 + (1 if splits > 1 else 0)
 
 
+def attention_launches(T: int, k: int, sms: int) -> int:
+    """Kernels one dsa_sparse_mla_attn launches: attention, and the split merge."""
+    ntiles = (k + 127) // 128
+    return 1 + (1 if max(1, min(16, ntiles, sms // max(T, 1))) > 1 else 0)
+
+
 def rank_seed(cfg: int, rank: int) -> int:
     """Each rank draws its own replica batch (weak scaling)."""
     return cfg + 7919 * rank
@@ -243,8 +257,50 @@ def run_ours(args, rank, world, dist):
     ws = B.workspace(B.DSA_OP_FORWARD, T, max_n, k, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    # IndexShare (N^2, section "IndexShare"): a group of L layers runs the indexer
+    # and the top-k once (the full layer) and L - 1 shared layers attend over the
+    # same index set with their own queries and latent caches.
+    L = max(1, args.indexshare)
+    shared = [wl.make_shared_layer_torch(c, l, dev, seed=rank_seed(cfg, rank)) for l in range(1, L)]
+    mla_ws = B.workspace(B.DSA_OP_SPARSE_MLA, T, max_n, k, device=dev)
+    o_sh = [torch.empty_like(o) for _ in shared]
+    lse_sh = [torch.empty_like(lse) for _ in shared]
+
+    def full_layer():
         B.dsa_forward(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, max_n, k, wl.SCALE, o, lse, idx, ws, stream)
+
+    # Dense + sparse ("GLM-5.2's DSA architecture: how dense and sparse attention
+    # split the work", section "DSA's core design"): the selection, then both
+    # attention branches (window of W positions, selected set) fused per head.
+    W = args.dense_window
+    if W > 0:
+        gate = torch.full((T, 64), 0.5, dtype=torch.float32, device=dev)   # the caller's fusion weights
+        ds_ws = B.workspace(B.DSA_OP_DENSE_SPARSE, T, 0, 0, device=dev)
+        if forward_streams(T, max_n):
+            sel_ws0 = B.workspace(B.DSA_OP_INDEXER_TOPK, T, max_n, k, device=dev)
+
+            def select():
+                B.dsa_indexer_topk(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, max_n, k, idx, sel_ws0, stream)
+        else:
+            plan_ws0 = B.workspace(B.DSA_OP_INDEXER, T, max_n, k, device=dev)
+            scores0 = torch.empty((T, (max_n + 3) // 4 * 4), dtype=torch.float32, device=dev)
+
+            def select():
+                B.dsa_indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, scores0, plan_ws0, stream)
+                B.dsa_topk(scores0, c.n_vis, k, idx, stream)
+
+        def dense_sparse():
+            B.dsa_dense_sparse_attn(c.q, c.kv, c.kv_start, c.n_vis, idx, W, gate, wl.SCALE, o, None, None, ds_ws,
+                                    stream)
+
+    def step():
+        if W > 0:
+            select()
+            dense_sparse()
+            return
+        full_layer()
+        for (q_l, kv_l), o_l, lse_l in zip(shared, o_sh, lse_sh):
+            B.dsa_sparse_mla_attn(q_l, kv_l, c.kv_start, idx, wl.SCALE, o_l, lse_l, mla_ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -287,7 +343,6 @@ def run_ours(args, rank, world, dist):
     streams = forward_streams(T, max_n)
     nb = max(3, min(args.steps, 50))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
-    mla_ws = B.workspace(B.DSA_OP_SPARSE_MLA, T, max_n, k, device=dev)
     wm = work_model(n_vis_h, c.kv_start.cpu().numpy())
     pk = peaks()
     workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
@@ -340,15 +395,55 @@ def run_ours(args, rank, world, dist):
                     "frac": v["frac"]} for kk, v in per_kernel.items()}
     step_rf = roofline_of("dsa_forward step", ms_step, wm["step_bytes"], wm["step_flops"], pk)
 
+    plain = (L == 1 and W == 0)
+    dense_info = None
+    if W > 0:
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_t = max(3, min(args.steps, 200))
+        a.record(stream)
+        for _ in range(n_t):
+            dense_sparse()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        B.dsa_sync_status(stream)
+        dense_info = {"window": W, "gate": "0.5 for every (row, head)",
+                      "dense_sparse_attention_ms": round(a.elapsed_time(b) / n_t, 4),
+                      "sparse_attention_only_ms": round(t_att, 4)}
+        workload += f"_dense{W}"
+    indexshare = None
+    if L > 1:
+        # the full layer alone, and one shared layer's attention, timed the same way
+        def timed(fn, n):
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(n):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) / n
+        n_t = max(3, min(args.steps, 200))
+        t_full = timed(full_layer, n_t)
+        q1, kv1 = shared[0]
+        t_shared = timed(lambda: B.dsa_sparse_mla_attn(q1, kv1, c.kv_start, idx, wl.SCALE, o_sh[0], lse_sh[0],
+                                                      mla_ws, stream), n_t)
+        B.dsa_sync_status(stream)
+        indexshare = {"layers": L, "full_layers": 1, "shared_layers": L - 1, "group_ms": round(ms_step, 4),
+                      "full_layer_ms": round(t_full, 4), "shared_layer_ms": round(t_shared, 4),
+                      "shared_layer_tokens_per_s": round(whole_job_rate(T, world, t_shared), 1),
+                      "unshared_group_ms_estimate": round(L * t_full, 4)}
+        workload += f"_indexshare{L}"
+
     # ---- end to end through dsa_forward with host buffers
     e2e = None
-    if not args.skip_e2e:
+    if not args.skip_e2e and plain:
         e2e = run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist)
         if e2e is not None:
             e2e["value"] = round(whole_job_rate(T, world, e2e.pop("ms_per_step")), 1)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu:
+    if rank == 0 and world == 1 and not args.skip_cpu and plain:
         cpu = cpu_baseline(c, o, lse, idx, args)
 
     value = whole_job_rate(T, world, ms_step)
@@ -366,10 +461,18 @@ def run_ours(args, rank, world, dist):
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step(T, k, streams, torch.cuda.get_device_properties(dev).multi_processor_count)
+        "gpu_launches": (launches_per_step(T, k, streams, torch.cuda.get_device_properties(dev).multi_processor_count)
+                         + (L - 1) * attention_launches(T, k, torch.cuda.get_device_properties(dev).multi_processor_count))
         * args.steps,
         "clocks": clocks,
     }
+    if indexshare is not None:
+        out["indexshare"] = indexshare
+    if dense_info is not None:
+        out["dense_sparse"] = dense_info
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        # dsa_forward's kernels (its attention is the sparse branch), the dense branch, window indices, fusion
+        out["gpu_launches"] = (launches_per_step(T, k, streams, sms) + attention_launches(T, W, sms) + 2) * args.steps
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -532,6 +635,12 @@ def main():
     ap.add_argument("--scale", type=int, default=1, help="shrink contexts by this factor (small captures)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--dense-window", type=int, default=0,
+                    help="time the dense + sparse layer instead: selection, then attention over the selected set "
+                         "and over a window of W positions, fused per head (default 0: off)")
+    ap.add_argument("--indexshare", type=int, default=1,
+                    help="layers per IndexShare group: one step = one full layer (indexer, top-k, attention) "
+                         "+ L-1 layers attending over its index set (default 1: no sharing)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -79,7 +79,8 @@ enum dsa_op {
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_MLA = 2,
   DSA_OP_FORWARD = 3,
-  DSA_OP_INDEXER_TOPK = 4
+  DSA_OP_INDEXER_TOPK = 4,
+  DSA_OP_DENSE_SPARSE = 5
 };
 
 /*
@@ -152,6 +153,33 @@ DSA_API int dsa_topk(const float* scores, int64_t score_ld, const int32_t* n_vis
 DSA_API int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
                         const int32_t* idx, int T, int topk, float scale, float* o_lat, float* lse, void* ws,
                         size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Dense + sparse attention, the two branches of a DSA layer fused ("GLM-5.2's
+ * DSA architecture: how dense and sparse attention split the work", section
+ * "DSA's core design: dense and sparse side by side": local dense attention over
+ * a sliding window next to the current token, global sparse attention over the
+ * selected top-k positions, outputs fused inside the layer with learned
+ * weights).  For row i with n = n_vis[i], the attention of dsa_sparse_mla_attn
+ * is taken twice:
+ *     o_sparse over idx[i, 0:topk]
+ *     o_dense  over the window positions n - window .. n - 1 (those >= 0)
+ *     o_lat[i,h,:] = gate[i,h] * o_dense[i,h,:] + (1 - gate[i,h]) * o_sparse[i,h,:]
+ * The pages give neither the window length nor the fusion formula: the window
+ * is the caller's, and the learned fusion is read as a per-(row, head) weight
+ * gate in [0, 1] supplied by the caller.
+ *
+ *  q, kv, kv_start, idx, scale, o_lat   as for dsa_sparse_mla_attn
+ *  n_vis       [T] int32 (device), n_vis[i] >= 1 (rows with n_vis < 1: status bit, -1 window)
+ *  window      1 <= window <= 2048
+ *  gate        [T,64] fp32 (device)
+ *  lse_dense, lse_sparse  [T,64] fp32 or NULL: each branch's log-sum-exp
+ *  ws          >= dsa_workspace_size(DSA_OP_DENSE_SPARSE, T, 0, 0) bytes, 256-byte aligned
+ */
+DSA_API int dsa_dense_sparse_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows,
+                                  const int64_t* kv_start, const int32_t* n_vis, const int32_t* idx, int T, int topk,
+                                  int window, const float* gate, float scale, float* o_lat, float* lse_dense,
+                                  float* lse_sparse, void* ws, size_t ws_bytes, dsa_stream_t stream);
 
 /*
  * Indexer and top-k fused, without a score matrix ("2026 LLM architecture

@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_UNSUPPORTED, DSA_ERR_BAD_ROW = range(7)
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD, DSA_OP_INDEXER_TOPK = range(5)
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD, DSA_OP_INDEXER_TOPK, DSA_OP_DENSE_SPARSE = range(6)
 INDEX_HEADS, INDEX_DIM, HEADS, LATENT, ROPE, ROW, MAX_TOPK = 32, 128, 64, 512, 64, 576, 2048
 NOALLOC_MAX_ROWS = 8192
 
@@ -50,6 +50,8 @@ def lib():
         L.dsa_indexer_topk.argtypes = [P, P, P, I64, P, P, I, I64, I, P, P, SZ, P]
         L.dsa_indexer_topk.restype = I
         L.dsa_indexer_scores_noalloc.argtypes = [P, P, P, I64, P, P, I, P, I64, P]
+        L.dsa_dense_sparse_attn.argtypes = [P, P, I64, P, P, P, I, I, I, P, F, P, P, P, P, SZ, P]
+        L.dsa_dense_sparse_attn.restype = I
         L.dsa_indexer_scores_noalloc.restype = I
         L.dsa_last_error_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I
@@ -163,6 +165,27 @@ def dsa_sparse_mla_attn(q, kv, kv_start, idx, scale, o_lat, lse=None, ws=None, s
     _check(lib().dsa_sparse_mla_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(kv_start), _ptr(idx), T, topk,
                                      float(scale), _ptr(o_lat), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
                                      _stream(stream)))
+
+
+def dsa_dense_sparse_attn(q, kv, kv_start, n_vis, idx, window, gate, scale, o_lat, lse_dense=None, lse_sparse=None,
+                          ws=None, stream=None):
+    import torch
+    T, topk = idx.shape
+    _need(q, torch.bfloat16, (T, HEADS, ROW), "q")
+    _need(kv, torch.bfloat16, None, "kv")
+    _need(kv_start, torch.int64, (T,), "kv_start")
+    _need(n_vis, torch.int32, (T,), "n_vis")
+    _need(idx, torch.int32, (T, topk), "idx")
+    _need(gate, torch.float32, (T, HEADS), "gate")
+    _need(o_lat, torch.float32, (T, HEADS, LATENT), "o_lat")
+    for t, nm in ((lse_dense, "lse_dense"), (lse_sparse, "lse_sparse")):
+        if t is not None:
+            _need(t, torch.float32, (T, HEADS), nm)
+    if ws is not None:
+        _need(ws, torch.uint8, None, "ws")
+    _check(lib().dsa_dense_sparse_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(kv_start), _ptr(n_vis), _ptr(idx), T, topk,
+                                       int(window), _ptr(gate), float(scale), _ptr(o_lat), _ptr(lse_dense),
+                                       _ptr(lse_sparse), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def dsa_forward(q_I, w, k_I, q, kv, kv_start, n_vis, max_n_vis, topk, scale, o_lat, lse, idx_out, ws, stream=None):

@@ -15,6 +15,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+#include "dense_sparse.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
@@ -182,6 +183,13 @@ size_t ws_forward(int T, int64_t max_n_vis, int topk) {
   return ws_indexer(T) + sel + align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
 }
 
+// dense + sparse: window index rows (up to DSA_MAX_TOPK wide), the dense branch's
+// output, then the attention partials
+size_t ws_dense_sparse(int T) {
+  return align_up(size_t(T) * DSA_MAX_TOPK * 4, 256) + align_up(size_t(T) * DSA_HEADS * DSA_LATENT * 4, 256) +
+         ws_mla(T, DSA_MAX_TOPK);
+}
+
 int pick_qmax(int T) {
   const char* s = std::getenv("DSA_INDEXER_QMAX");
   if (s && *s) {
@@ -272,6 +280,7 @@ size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
     case DSA_OP_SPARSE_MLA: return ws_mla(T, topk);
     case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
     case DSA_OP_INDEXER_TOPK: return ws_indexer(T) + ws_select(T);
+    case DSA_OP_DENSE_SPARSE: return ws_dense_sparse(T);
     default: return 0;
   }
 }
@@ -335,6 +344,50 @@ int dsa_sparse_mla_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_row
   dsa::MlaLaunch p{q,     kv,  cache_rows, kv_start, idx, T, topk, scale, o_lat, lse, static_cast<float*>(ws),
                    ws ? ws_bytes : 0, dev->sm_count, wait_limit_ns(), stream};
   return run_sparse_mla(p);
+}
+
+int dsa_dense_sparse_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
+                          const int32_t* n_vis, const int32_t* idx, int T, int topk, int window, const float* gate,
+                          float scale, float* o_lat, float* lse_dense, float* lse_sparse, void* ws, size_t ws_bytes,
+                          dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_INVALID_ARG, "topk must lie in [1, %d]", DSA_MAX_TOPK);
+  if (window < 1 || window > DSA_MAX_TOPK)
+    return fail(DSA_ERR_INVALID_ARG, "window must lie in [1, %d]", DSA_MAX_TOPK);
+  if (T == 0) return DSA_OK;
+  if (!q || !kv || !n_vis || !idx || !gate || !o_lat || !ws)
+    return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o_lat, 16) || !aligned(n_vis, 4) || !aligned(idx, 4) ||
+      !aligned(gate, 4) || !aligned(lse_dense, 4) || !aligned(lse_sparse, 4))
+    return fail(DSA_ERR_INVALID_ARG, "q, kv, o_lat must be 16-byte aligned; n_vis, idx, gate, lse 4-byte aligned");
+  if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (int64_t(T) * DSA_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
+  const size_t need = ws_dense_sparse(T);
+  if (ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, need);
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int32_t* idx_w = reinterpret_cast<int32_t*>(base);
+  float* o_dense = reinterpret_cast<float*>(base + align_up(size_t(T) * DSA_MAX_TOPK * 4, 256));
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(o_dense) +
+                                         align_up(size_t(T) * DSA_HEADS * DSA_LATENT * 4, 256));
+  const size_t part_bytes = ws_mla(T, DSA_MAX_TOPK);
+  // sparse branch into o_lat
+  dsa::MlaLaunch ps{q,          kv,         cache_rows,   kv_start,      idx,           T,     topk, scale,
+                    o_lat,      lse_sparse, part,         part_bytes,    dev->sm_count, wait_limit_ns(), stream};
+  if ((rc = run_sparse_mla(ps))) return rc;
+  // dense branch over the window, into the workspace
+  cudaError_t e = dsa::launch_window_idx(n_vis, T, window, idx_w, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "window index launch");
+  dsa::MlaLaunch pd{q,          kv,         cache_rows,   kv_start,      idx_w,         T,     window, scale,
+                    o_dense,    lse_dense,  part,         part_bytes,    dev->sm_count, wait_limit_ns(), stream};
+  if ((rc = run_sparse_mla(pd))) return rc;
+  e = dsa::launch_fuse(o_lat, o_dense, gate, T, dev->sm_count, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fusion launch");
+  return DSA_OK;
 }
 
 int dsa_indexer_topk(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,

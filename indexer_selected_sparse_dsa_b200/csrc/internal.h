@@ -105,6 +105,10 @@ struct MlaLaunch {
 };
 cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q);
 
+// ------------------------------------------------------------------ dense + sparse branches
+cudaError_t launch_window_idx(const int32_t* n_vis, int T, int window, int32_t* idx_w, cudaStream_t stream);
+cudaError_t launch_fuse(float* o, const float* o_dense, const float* gate, int T, int sm_count, cudaStream_t stream);
+
 // Shared-memory opt-in sizes, set once per device.
 cudaError_t prepare_indexer();
 cudaError_t prepare_sparse_mla();

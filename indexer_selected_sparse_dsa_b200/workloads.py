@@ -327,3 +327,30 @@ def case_to_host(c: Case, rows=None) -> Case:
     return Case(u16(c.q_I[sel]), u16(c.w[sel]), u16(c.k_I), u16(c.q[sel]), u16(c.kv),
                 ks.cpu().numpy().astype(np.int64), (c.n_vis[sel] if rows is not None else c.n_vis).cpu().numpy().astype(np.int32),
                 c.plants[np.asarray(rows)] if rows is not None else c.plants, c.topk, c.name)
+
+
+def make_shared_layer_torch(c: Case, layer: int, device, seed: int = 0, chunk_rows: int = 1 << 20):
+    """Inputs of a further layer that shares ``c``'s indexer (IndexShare): its
+    own queries q [T,64,576] and latent cache kv [rows,576], drawn like ``c``'s
+    (N(0,1), bf16) from a seeded torch generator; the index set, kv_start and
+    n_vis are the full layer's."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(1000003 * (layer + 1) + seed)
+    q = torch.randn(tuple(c.q.shape), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    kv = torch.empty(tuple(c.kv.shape), dtype=torch.bfloat16, device=device)
+    L = kv.shape[0]
+    for r0 in range(0, L, chunk_rows):
+        r1 = min(L, r0 + chunk_rows)
+        kv[r0:r1] = torch.randn((r1 - r0, D_QK), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return q, kv
+
+
+def make_shared_layer_numpy(c: Case, layer: int, seed: int = 0):
+    """numpy (uint16 bf16 bits) counterpart of ``make_shared_layer_torch``."""
+    r = np.random.default_rng(1000003 * (layer + 1) + seed)
+    q = bf16_from_f32(r.standard_normal(c.q.shape).astype(np.float32))
+    kv = bf16_from_f32(r.standard_normal(c.kv.shape).astype(np.float32))
+    return q, kv
+

@@ -12,6 +12,8 @@ Functions (all inputs are bf16 bit patterns as uint16 arrays):
   topk(scores, n_vis, topk)                              -> int32 [T, topk]
   sparse_mla(q, kv, kv_start, idx, scale)                -> (o_lat f64 [T,64,512], lse f64 [T,64])
   forward(case or arrays, topk, scale)                   -> (o_lat, lse, idx)
+  dense_sparse(q, kv, kv_start, n_vis, idx, window, gate, scale)
+                                                         -> (o_lat, lse_dense, lse_sparse)
 """
 from __future__ import annotations
 
@@ -113,6 +115,26 @@ def forward(q_I, w, k_I, q, kv, kv_start, n_vis, k, scale, nthreads=NTHREADS):
     lib().oracle_forward(_p(q_I), _p(w), _p(k_I), _p(q), _p(kv), _p(kv_start), _p(n_vis), T, k,
                          float(scale), _p(o), _p(lse), _p(idx), nthreads)
     return o, lse, idx
+
+
+def window_indices(n_vis, window):
+    """The dense branch's positions: n - window .. n - 1 of each row, -1 where
+    negative (rows shorter than the window)."""
+    n = np.asarray(n_vis, np.int64)[:, None]
+    p = n - window + np.arange(window, dtype=np.int64)[None, :]
+    return np.where(p >= 0, p, -1).astype(np.int32)
+
+
+def dense_sparse(q, kv, kv_start, n_vis, idx, window, gate, scale, nthreads=NTHREADS):
+    """Dense + sparse DSA layer ("GLM-5.2's DSA architecture: how dense and sparse
+    attention split the work", section "DSA's core design"): local dense
+    attention over the last ``window`` visible positions and sparse attention over
+    ``idx``, fused per (row, head) with the caller's weight ``gate`` [T, 64]:
+    o = gate * o_dense + (1 - gate) * o_sparse.  Each branch is ``sparse_mla``."""
+    o_s, lse_s = sparse_mla(q, kv, kv_start, idx, scale, nthreads)
+    o_d, lse_d = sparse_mla(q, kv, kv_start, window_indices(n_vis, window), scale, nthreads)
+    g = np.asarray(gate, np.float64)[:, :, None]
+    return g * o_d + (1.0 - g) * o_s, lse_d, lse_s
 
 
 def forward_case(c, scale, nthreads=NTHREADS):

@@ -93,6 +93,15 @@ def test_host_validation_rejects_bad_arguments(L):
                        fake, z, z, fake, 1 << 30, z), B.DSA_ERR_INVALID_ARG)
     _err(L.dsa_forward(fake, fake, fake, fake, fake, 100, fake, fake, 4, 100, 16, ctypes.c_float(0.0625),
                        fake, z, z, fake, 256, z), B.DSA_ERR_WORKSPACE)
+    # dense + sparse: window out of range, null gate, workspace too small
+    ds = L.dsa_dense_sparse_attn
+    for window in (0, 2049):
+        _err(ds(fake, fake, 100, fake, fake, fake, 4, 16, window, fake, ctypes.c_float(0.0625), fake, z, z, fake,
+                1 << 30, z), B.DSA_ERR_INVALID_ARG)
+    _err(ds(fake, fake, 100, fake, fake, fake, 4, 16, 64, z, ctypes.c_float(0.0625), fake, z, z, fake, 1 << 30, z),
+         B.DSA_ERR_INVALID_ARG)
+    _err(ds(fake, fake, 100, fake, fake, fake, 4, 16, 64, fake, ctypes.c_float(0.0625), fake, z, z, fake, 256, z),
+         B.DSA_ERR_WORKSPACE)
 
 
 def test_empty_batch_is_a_no_op(L):
@@ -100,3 +109,5 @@ def test_empty_batch_is_a_no_op(L):
     assert L.dsa_topk(z, 8, z, 0, 16, z, z) == B.DSA_OK
     assert L.dsa_indexer_scores(z, z, z, 10, z, z, 0, z, 8, z, 0, z) == B.DSA_OK
     assert L.dsa_sparse_mla_attn(z, z, 10, z, z, 0, 16, ctypes.c_float(0.0625), z, z, z, 0, z) == B.DSA_OK
+    assert L.dsa_dense_sparse_attn(z, z, 10, z, z, z, 0, 16, 64, z, ctypes.c_float(0.0625), z, z, z, z, 0,
+                                   z) == B.DSA_OK

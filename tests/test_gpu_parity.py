@@ -309,6 +309,61 @@ def test_forward_ragged_decode_scaled():
     _forward_check(wl.make_workload_numpy(3, scale=32))
 
 
+# ---------------------------------------------------------------------------- IndexShare
+
+@pytest.mark.parametrize("split", [False, True])
+def test_indexshare_shared_layers_match_oracle(split):
+    """A group of four layers (N^2, section "IndexShare"): the full layer runs the
+    whole step; three further layers attend over its index set with their own
+    queries and latent caches and must match the oracle's attention on that set."""
+    import torch
+    c = wl.make_case_numpy([6000], [(0, 6000), (0, 5000), (0, 2100), (0, 900), (0, 1)], seed=71)
+    d = to_dev(c)
+    o0, lse0, idx = gpu_forward(d, 6000, 2048)
+    o0_ref, lse0_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, wl.SCALE)
+    assert_attention_close(o0, lse0, o0_ref, lse0_ref)
+    for layer in (1, 2, 3):
+        q_l, kv_l = wl.make_shared_layer_numpy(c, layer)
+        dl = dict(d)
+        dl["q"] = torch.from_numpy(q_l.view(np.int16)).view(torch.bfloat16).cuda()
+        dl["kv"] = torch.from_numpy(kv_l.view(np.int16)).view(torch.bfloat16).cuda()
+        o, lse = gpu_attention(dl, idx, split=split)
+        o_ref, lse_ref = oracle.sparse_mla(q_l, kv_l, c.kv_start, idx, wl.SCALE)
+        assert_attention_close(o, lse, o_ref, lse_ref)
+        assert not np.allclose(o, o0)   # the layers differ; only the index set is shared
+
+
+# ---------------------------------------------------------------------------- dense + sparse branches
+
+@pytest.mark.parametrize("window", [1, 128, 700, 2048])
+def test_dense_sparse_matches_oracle(window):
+    """Two branches fused by a per-head gate ("GLM-5.2's DSA architecture: how dense
+    and sparse attention split the work", section "DSA's core design")."""
+    import torch
+    c = wl.make_case_numpy([3000], [(0, 3000), (0, 2500), (0, 1000), (0, 130), (0, 1)], seed=93, n_plant=0)
+    r = np.random.default_rng(94 + window)
+    k = 2048
+    idx = np.full((c.T, k), -1, np.int32)
+    for i, n in enumerate(c.n_vis):
+        m = min(k, int(n)) - (100 if n > 2100 else 0)
+        idx[i, :m] = np.sort(r.choice(int(n), m, replace=False))
+    gate = r.uniform(0, 1, (c.T, 64)).astype(np.float32)
+    gate[1] = 0.0
+    gate[2] = 1.0
+    d = to_dev(c)
+    o = torch.full((c.T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse_d = torch.full((c.T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    lse_s = torch.full((c.T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    ws = B.workspace(B.DSA_OP_DENSE_SPARSE, c.T, 0, 0)
+    B.dsa_dense_sparse_attn(d["q"], d["kv"], d["kv_start"], d["n_vis"], torch.from_numpy(idx).cuda(), window,
+                            torch.from_numpy(gate).cuda(), SCALE, o, lse_d, lse_s, ws)
+    B.dsa_sync_status()
+    o_ref, ld_ref, ls_ref = oracle.dense_sparse(c.q, c.kv, c.kv_start, c.n_vis, idx, window, gate.astype(np.float64),
+                                                SCALE)
+    assert_attention_close(o.cpu().numpy(), lse_d.cpu().numpy(), o_ref, ld_ref)
+    assert_attention_close(o.cpu().numpy(), lse_s.cpu().numpy(), o_ref, ls_ref)
+
+
 # ---------------------------------------------------------------------------- streamed selection
 
 STREAM_CASES = {

@@ -296,3 +296,62 @@ def test_planted_positions_are_recalled():
         p = c.plants[i][c.plants[i] >= 0]
         assert p.size > 0
         assert np.isin(p, idx[i]).all()
+
+
+# ---------------------------------------------------------------------------- dense + sparse branches
+# ("GLM-5.2's DSA architecture: how dense and sparse attention split the work",
+# section "DSA's core design": a sliding-window dense branch next to the sparse
+# branch, fused per head by learned weights, here a caller-supplied gate.)
+
+def _window_reference(qi, kv, ks, n, window, scale):
+    """Dense attention of one row over its last `window` visible positions, with
+    scipy's softmax / logsumexp (no oracle code)."""
+    lo = max(0, n - window)
+    K = f32(kv[ks + lo:ks + n])
+    S = (f32(qi) @ K.T) * scale
+    return softmax(S, axis=1) @ K[:, :512], logsumexp(S, axis=1)
+
+
+def test_dense_sparse_gate_extremes_are_the_branches():
+    r = np.random.default_rng(91)
+    L = 700
+    kv = wl.bf16_from_f32(r.standard_normal((L + 50, 576)).astype(np.float32))
+    q = wl.bf16_from_f32(r.standard_normal((4, 64, 576)).astype(np.float32))
+    kv_start = np.array([50, 50, 0, 10], np.int64)
+    n_vis = np.array([700, 300, 5, 640], np.int32)
+    idx = np.full((4, 96), -1, np.int32)
+    for i, n in enumerate(n_vis):
+        m = min(96, int(n))
+        idx[i, :m] = np.sort(r.choice(int(n), m, replace=False))
+    for window in (1, 64, 128, 1000):
+        o1, ld, ls = oracle.dense_sparse(q, kv, kv_start, n_vis, idx, window, np.ones((4, 64)), 1 / 16)
+        o0, ld0, ls0 = oracle.dense_sparse(q, kv, kv_start, n_vis, idx, window, np.zeros((4, 64)), 1 / 16)
+        os_, lss = oracle.sparse_mla(q, kv, kv_start, idx, 1 / 16)
+        assert np.array_equal(o0, os_) and np.array_equal(ls, lss)   # gate 0: the sparse branch alone
+        for i, n in enumerate(n_vis):
+            ro, rl = _window_reference(q[i], kv, int(kv_start[i]), int(n), window, 1 / 16)
+            assert np.max(np.abs(o1[i] - ro)) < 1e-12                 # gate 1: the window alone
+            assert np.max(np.abs(ld[i] - rl)) < 1e-12
+
+
+def test_dense_sparse_gate_mixes_per_head():
+    r = np.random.default_rng(92)
+    L = 400
+    kv = wl.bf16_from_f32(r.standard_normal((L, 576)).astype(np.float32))
+    q = wl.bf16_from_f32(r.standard_normal((2, 64, 576)).astype(np.float32))
+    kv_start = np.zeros(2, np.int64)
+    n_vis = np.array([400, 250], np.int32)
+    idx = np.stack([np.sort(r.choice(int(n), 64, replace=False)) for n in n_vis]).astype(np.int32)
+    gate = r.uniform(0, 1, (2, 64))
+    o, _, _ = oracle.dense_sparse(q, kv, kv_start, n_vis, idx, 32, gate, 1 / 16)
+    os_, _ = oracle.sparse_mla(q, kv, kv_start, idx, 1 / 16)
+    for i, n in enumerate(n_vis):
+        ro, _ = _window_reference(q[i], kv, 0, int(n), 32, 1 / 16)
+        for h in (0, 17, 63):
+            want = gate[i, h] * ro[h] + (1 - gate[i, h]) * os_[i, h]
+            assert np.max(np.abs(o[i, h] - want)) < 1e-12
+    # a window covering the whole context is full dense attention
+    o_full, _, _ = oracle.dense_sparse(q, kv, kv_start, n_vis, idx, 2048, np.ones((2, 64)), 1 / 16)
+    for i, n in enumerate(n_vis):
+        ro, _ = dense_reference(q[i], kv, int(n), 1 / 16)
+        assert np.max(np.abs(o_full[i] - ro)) < 1e-12
