@@ -255,7 +255,9 @@ def run_ours(args, rank, world, dist):
     lse = torch.empty((T, 64), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     ws = B.workspace(B.DSA_OP_FORWARD, T, max_n, k, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    # a stream of our own: the timed steps can be captured into a CUDA graph on it
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.Stream(dev)
 
     # IndexShare (N^2, section "IndexShare"): a group of L layers runs the indexer
     # and the top-k once (the full layer) and L - 1 shared layers attend over the
@@ -306,16 +308,33 @@ def run_ours(args, rank, world, dist):
         step()
     B.dsa_sync_status(stream)
 
-    # ---- timed region: exactly K steps of dsa_forward
+    # One step captured as a CUDA graph (the library's calls only enqueue kernels
+    # and memsets on the stream), replayed K times: no host launch gaps.
+    run, graph_note = step, None
+    if args.graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    step()
+            torch.cuda.synchronize(dev)
+            run = g.replay
+        except Exception as e:  # capture refused: time the eager launches instead
+            torch.cuda.synchronize(dev)
+            graph_note = f"eager launches (graph capture failed: {type(e).__name__})"
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: exactly K steps
     sampler = ClockSampler(bus_id_of(dev))
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            run()
+        ev1.record(stream)
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
@@ -328,10 +347,11 @@ def run_ours(args, rank, world, dist):
         # timed region shorter than the sampling interval: sample an equal-load loop
         s2 = ClockSampler(bus_id_of(dev))
         t_end = time.time() + 1.0
-        while time.time() < t_end:
-            for _ in range(20):
-                step()
-            torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            while time.time() < t_end:
+                for _ in range(20):
+                    run()
+                torch.cuda.synchronize(dev)
         s2.stop()
         clocks = s2.summary()
         if clocks is not None:
@@ -465,6 +485,7 @@ def run_ours(args, rank, world, dist):
                          + (L - 1) * attention_launches(T, k, torch.cuda.get_device_properties(dev).multi_processor_count))
         * args.steps,
         "clocks": clocks,
+        "launch": graph_note or ("one CUDA graph per step (captured dsa_forward)" if args.graph else "eager launches"),
     }
     if indexshare is not None:
         out["indexshare"] = indexshare
@@ -498,7 +519,7 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
     bi = sum(v.numel() * v.element_size() for v in h.values())
     bo = o_h.numel() * 4 + lse_h.numel() * 4
 
-    def step():
+    def step_on_stream():
         for kk in h:
             d[kk].copy_(h[kk], non_blocking=True)
         c.k_I.index_copy_(0, d["rows"], d["k_new"])
@@ -507,6 +528,10 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
                       o, lse, idx, ws, stream)
         o_h.copy_(o, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
+
+    def step():
+        with torch.cuda.stream(stream):   # copies, cache update and dsa_forward in one stream order
+            step_on_stream()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -635,6 +660,8 @@ def main():
     ap.add_argument("--scale", type=int, default=1, help="shrink contexts by this factor (small captures)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time eager launches instead of replaying the step captured as a CUDA graph")
     ap.add_argument("--dense-window", type=int, default=0,
                     help="time the dense + sparse layer instead: selection, then attention over the selected set "
                          "and over a window of W positions, fused per head (default 0: off)")

@@ -22,6 +22,7 @@ namespace {
 // idx_w[i, j] = n_vis[i] - window + j, or -1 where that is negative (rows shorter
 // than the window); ascending, like every index row of the library.
 __global__ void window_idx_kernel(const int32_t* __restrict__ n_vis, int T, int window, int32_t* __restrict__ idx_w) {
+  pdl_wait();
   const int i = blockIdx.x;
   const int n = n_vis[i];
   if (n < 1 && threadIdx.x == 0) raise_status(kStatusBadRow);
@@ -35,6 +36,7 @@ __global__ void window_idx_kernel(const int32_t* __restrict__ n_vis, int T, int 
 // o[i,h,:] = gate[i,h] * o_dense[i,h,:] + (1 - gate[i,h]) * o[i,h,:], in place.
 __global__ void fuse_kernel(float* __restrict__ o, const float* __restrict__ o_dense, const float* __restrict__ gate,
                             long long n4) {
+  pdl_wait();
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n4; v += (long long)gridDim.x * blockDim.x) {
     const float g = gate[(v * 4) >> 9];  // 512 latent dims per (row, head)
     const float4 d = reinterpret_cast<const float4*>(o_dense)[v];
@@ -51,8 +53,7 @@ __global__ void fuse_kernel(float* __restrict__ o, const float* __restrict__ o_d
 
 cudaError_t launch_window_idx(const int32_t* n_vis, int T, int window, int32_t* idx_w, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
-  window_idx_kernel<<<T, 256, 0, stream>>>(n_vis, T, window, idx_w);
-  return cudaGetLastError();
+  return launch_pdl(window_idx_kernel, dim3(unsigned(T)), dim3(256), 0, stream, 1, n_vis, T, window, idx_w);
 }
 
 cudaError_t launch_fuse(float* o, const float* o_dense, const float* gate, int T, int sm_count, cudaStream_t stream) {
@@ -60,8 +61,7 @@ cudaError_t launch_fuse(float* o, const float* o_dense, const float* gate, int T
   const long long n4 = (long long)T * 64 * 512 / 4;
   const long long want = (n4 + 255) / 256;
   const int grid = int(want < 8LL * sm_count ? want : 8LL * sm_count);
-  fuse_kernel<<<grid, 256, 0, stream>>>(o, o_dense, gate, n4);
-  return cudaGetLastError();
+  return launch_pdl(fuse_kernel, dim3(unsigned(grid)), dim3(256), 0, stream, 1, o, o_dense, gate, n4);
 }
 
 }  // namespace dsa

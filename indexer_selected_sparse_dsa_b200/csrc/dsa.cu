@@ -264,6 +264,16 @@ int run_indexer(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int
 
 }  // namespace
 
+namespace dsa {
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("DSA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+}  // namespace dsa
+
 extern "C" {
 
 int dsa_abi_version(void) { return 1; }

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(const int64_t* __res
   __shared__ long long sc_l[33];
   __shared__ int carry_seg_s;
   const int tid = threadIdx.x;
+  pdl_wait();  // inputs and the plan buffer may belong to the previous kernel
   for (int i = tid; i < T; i += blockDim.x) {
     PlanTile z;
     z.q0 = 0;
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(1024) indexer_redo_plan_kernel(const int* __re
                                                                  PlanHeader* __restrict__ hdr,
                                                                  PlanTile* __restrict__ tiles) {
   __shared__ long long sc_l[33];
+  pdl_wait();
   const int n = redo[0];
   long long carry = 0;
   for (int base = 0; base < n; base += blockDim.x) {
@@ -317,6 +319,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // everything above touched shared memory and TMEM only
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -653,6 +656,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
   }
 
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -675,9 +679,9 @@ cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUt
   using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
   auto* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<const PlanTile*>(reinterpret_cast<const uint8_t*>(p.plan) + sizeof(PlanHeader));
-  indexer_kernel<QMAX, STAGES, QBUF, STREAM><<<p.grid, kIdxThreads, L::kAlloc, p.stream>>>(
-      tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, p.stream_out, WaitLimit{p.wait_ns});
-  return cudaGetLastError();
+  return launch_pdl(indexer_kernel<QMAX, STAGES, QBUF, STREAM>, dim3(p.grid), dim3(kIdxThreads), L::kAlloc,
+                    p.stream, 1, tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, p.stream_out,
+                    WaitLimit{p.wait_ns});
 }
 
 }  // namespace
@@ -701,17 +705,17 @@ cudaError_t launch_indexer(const IndexerLaunch& p, const CUtensorMap& tmap_k, co
   }
   auto* hdr = reinterpret_cast<PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<PlanTile*>(reinterpret_cast<uint8_t*>(p.plan) + sizeof(PlanHeader));
-  indexer_plan_kernel<<<1, 1024, 0, p.stream>>>(p.kv_start, p.n_vis, p.T, p.qmax, p.score_ld, p.cache_rows, hdr,
-                                                tiles);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(indexer_plan_kernel, dim3(1), dim3(1024), 0, p.stream, 1, p.kv_start, p.n_vis, p.T,
+                             p.qmax, p.score_ld, p.cache_rows, hdr, tiles);
   if (e != cudaSuccess) return e;
   if (p.streaming) {
     if (p.qmax != 8 || p.sweep != kSweepWave) return cudaErrorInvalidValue;
     if ((e = launch_main<8, 4, 1, true>(p, tmap_k, tmap_q)) != cudaSuccess) return e;
     // queries whose seeded threshold let too few keys through: sweep them again,
     // unseeded (an empty list costs one short launch, no host round trip)
-    indexer_redo_plan_kernel<<<1, 1024, 0, p.stream>>>(p.stream_out.redo, p.kv_start, p.n_vis, hdr, tiles);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(indexer_redo_plan_kernel, dim3(1), dim3(1024), 0, p.stream, 1, p.stream_out.redo,
+                        p.kv_start, p.n_vis, hdr, tiles)) != cudaSuccess)
+      return e;
     IndexerLaunch p2 = p;
     p2.stream_out.sample_units = 0;
     return launch_main<8, 4, 1, true>(p2, tmap_k, tmap_q);

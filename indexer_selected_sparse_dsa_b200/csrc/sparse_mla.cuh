@@ -192,7 +192,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   const int ntiles_row = (topk + kTileKeys - 1) / kTileKeys;
   const int t_first = sp * tiles_per_split;
   const int ntiles = max(0, min(ntiles_row, t_first + tiles_per_split) - t_first);
-  const long long ks = kv_start[i];
   const int32_t* irow = idx + (long long)i * topk;
 
   if (threadIdx.x == 0) {
@@ -222,6 +221,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // everything above touched shared memory and TMEM only
+  const long long ks = kv_start[i];
 
   if (warp < 4) {
     // ---------------------------------------------------------------- producers (warps 0..3)
@@ -535,6 +536,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
     }
   }
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -554,6 +556,7 @@ __global__ void __launch_bounds__(kCombineThreads) sparse_mla_combine_kernel(con
                                                                              float* __restrict__ lse) {
   __shared__ float wgt[16][kCombineHeads];
   __shared__ float inv_den[kCombineHeads];
+  pdl_wait();
   const int groups = 64 / kCombineHeads;
   const int i = blockIdx.x / groups;
   const int h0 = (blockIdx.x - i * groups) * kCombineHeads;
@@ -618,14 +621,12 @@ cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q) {
   const int per = (ntiles + splits - 1) / splits;
   splits = (ntiles + per - 1) / per;  // no split without tiles
   if (int64_t(p.T) * splits > INT32_MAX) return cudaErrorInvalidValue;
-  sparse_mla_kernel<<<p.T * splits, kMlaThreads, kSmemAlloc, p.stream>>>(
-      p.kv, tmap_q, p.cache_rows, p.kv_start, p.idx, p.topk, scale_log2, p.o_lat, p.lse, splits, per, p.part,
-      WaitLimit{p.wait_ns});
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(sparse_mla_kernel, dim3(unsigned(p.T * splits)), dim3(kMlaThreads), kSmemAlloc, p.stream, 1,
+                             p.kv, tmap_q, p.cache_rows, p.kv_start, p.idx, p.topk, scale_log2, p.o_lat, p.lse, splits,
+                             per, p.part, WaitLimit{p.wait_ns});
   if (e != cudaSuccess || splits == 1) return e;
-  sparse_mla_combine_kernel<<<p.T * (64 / kCombineHeads), kCombineThreads, 0, p.stream>>>(p.part, splits, p.o_lat,
-                                                                                         p.lse);
-  return cudaGetLastError();
+  return launch_pdl(sparse_mla_combine_kernel, dim3(unsigned(p.T * (64 / kCombineHeads))), dim3(kCombineThreads), 0,
+                    p.stream, 1, p.part, splits, p.o_lat, p.lse);
 }
 
 }  // namespace dsa

@@ -411,6 +411,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
                                                             int32_t* __restrict__ idx, int force_full, int split) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  pdl_wait();  // the scores come from the previous kernel
   // `split` CTAs (one cluster) per row; every branch below that returns early
   // depends on the row alone, so a cluster's CTAs take it together
   const int r = blockIdx.x / split;
@@ -604,6 +605,7 @@ __global__ void __launch_bounds__(kTopkThreads) stream_select_kernel(const uint3
                                                                      int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
+  pdl_wait();
   const int r = blockIdx.x;
   const int m = min(cnt[r], cap);
   if (m < 0) return;
@@ -631,9 +633,8 @@ cudaError_t prepare_topk() {
 cudaError_t launch_stream_select(const StreamOut& so, const int32_t* n_vis, int T, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   static_assert(kStreamCap <= kCandCap, "a streamed candidate buffer fits the shared candidate arrays");
-  stream_select_kernel<<<T, kTopkThreads, sizeof(TopkShared), stream>>>(so.cand_key, so.cand_pos, so.cnt_out, so.cap,
-                                                                       n_vis, so.topk, so.idx);
-  return cudaGetLastError();
+  return launch_pdl(stream_select_kernel, dim3(unsigned(T)), dim3(kTopkThreads), sizeof(TopkShared), stream, 1,
+                    so.cand_key, so.cand_pos, so.cnt_out, so.cap, n_vis, so.topk, so.idx);
 }
 
 cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk, int32_t* idx,
@@ -650,23 +651,8 @@ cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_
   }
   split = split >= 4 ? 4 : (split >= 2 ? 2 : 1);
   static_assert(4 * DSA_MAX_TOPK <= kCandCap, "rank 0 holds every CTA's top-k");
-  if (split == 1) {
-    topk_kernel<<<T, kTopkThreads, sizeof(TopkShared), stream>>>(scores, score_ld, n_vis, topk, idx, force_full, 1);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(T) * unsigned(split));
-  cfg.blockDim = dim3(kTopkThreads);
-  cfg.dynamicSmemBytes = sizeof(TopkShared);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = unsigned(split);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel, scores, score_ld, n_vis, topk, idx, force_full, split);
+  return launch_pdl(topk_kernel, dim3(unsigned(T) * unsigned(split)), dim3(kTopkThreads), sizeof(TopkShared), stream,
+                    unsigned(split), scores, score_ld, n_vis, topk, idx, force_full, split);
 }
 
 }  // namespace dsa
