@@ -11,9 +11,13 @@
 // head's dot product for 128 keys and up to 8 queries that share the
 // sequence.  Keys arrive by TMA (two 64-column boxes, 128-byte swizzle) into
 // a STAGES-deep ring; the query tile's q_I sits in its own buffer.  In the
-// epilogue each of 128 threads owns one key row: it reads that row's 32 head
-// columns per query from TMEM and reduces them with w into one fp32 score,
-// so the head reduction needs no cross-thread traffic.
+// epilogue a warp reads its 32 key rows x 32 head columns per query with the
+// 16x256b TMEM shape, so each lane sees 8 of the 32 heads (for 4 keys): the
+// lane keeps those 8 weights of each of its queries in registers for the
+// whole tile, weights and sums its 8 heads, and a 2-step shuffle
+// reduce-scatter over the 4 lanes that share a key row finishes the head sum
+// (one key per lane).  No weight is re-read from shared memory per key unit,
+// which leaves the shared-memory pipe to the tensor core's operand reads.
 //
 // Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
 // and MMA issuer, warps 2..9 = epilogue (two warps per TMEM lane quarter, each
@@ -420,7 +424,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // ---------------------------------------------------------------- epilogue (warps 2..9)
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;     // queries half, half + 2, half + 4, ...
-    const int row = quarter * 32 + lane;
+    // after the head reduce-scatter lane t holds key row t / 4 + 8 (t % 4) of the quarter
+    const int row = quarter * 32 + (lane >> 2) + 8 * (lane & 3);
+    const int hc = 2 * (lane & 3);        // this lane's heads: 8i + hc + {0, 1}, i < 4
     const int et = threadIdx.x - 64;      // 0 .. 32 * kEpiWarps - 1
     long long* thr_s = reinterpret_cast<long long*>(smem + L::kThrOff);
     int* cnt_s = reinterpret_cast<int*>(smem + L::kCntOff);
@@ -505,6 +511,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // shared memory only where they change (tile start, seeding, buffer checks).
     int nv_r[4];
     long long thr_r[4];
+    float wr[4][8];  // wr[j][2i + e] = w[query half + 2j, head 8i + hc + e]
     auto refresh = [&]() {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -535,6 +542,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         named_bar_sync(1, 32 * kEpiWarps);
         refresh();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int q = half + 2 * j;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) wr[j][e] = q < nq ? w_s[q * 32 + 8 * (e >> 1) + hc + (e & 1)] : 0.f;
+        }
         prev_tile = it.tile;
       }
       if (!mbar_wait(afull_bar(ab), aphase, lim, abort_flag)) break;
@@ -559,44 +572,39 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
         }
       };
-      // This warp's queries, two per TMEM wait: qi = half, half + 2 (then + 4, + 6).
+      // This warp's queries qi = half, half + 2, half + 4, half + 6, one TMEM wait each.
       // All scores are computed first and the accumulator is handed back to the
       // MMA warp before any is written or offered to a selection buffer.
       float sc[4];
 #pragma unroll
-      for (int it2 = 0; it2 < 2; ++it2) {
-        const int qi = half + 4 * it2, qj = qi + 2;
-        sc[2 * it2] = sc[2 * it2 + 1] = 0.f;
-        if (qi < nq) {
-          float v[64];
-          if (qj < nq) {
-            tmem_ld32x2_sync(tbase + uint32_t(qi * 32), tbase + uint32_t(qj * 32), v);
-          } else {
-            tmem_ld32_sync(tbase + uint32_t(qi * 32), v);
-          }
-          const float4* w0 = reinterpret_cast<const float4*>(w_s + qi * 32);
-          float a0 = 0.f, a1 = 0.f;
+      for (int j = 0; j < 4; ++j) {
+        const int qi = half + 2 * j;
+        sc[j] = 0.f;
+        if (qi < nq) {  // warp-uniform
+          float v[32];
+          const uint32_t tq = tbase + uint32_t(qi * 32);
+          tmem_ld16x256b_x4x2_sync(tq, tq + (16u << 16), v);
+          // p[r]: this lane's 8 heads of key row (lane / 4) + 8r
+          float p[4];
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 c = w0[h4];
-            a0 = fmaf(c.x, v[4 * h4], a0);
-            a0 = fmaf(c.y, v[4 * h4 + 1], a0);
-            a0 = fmaf(c.z, v[4 * h4 + 2], a0);
-            a0 = fmaf(c.w, v[4 * h4 + 3], a0);
-          }
-          if (qj < nq) {
-            const float4* w1 = reinterpret_cast<const float4*>(w_s + qj * 32);
+          for (int r = 0; r < 4; ++r) {
+            const float* x = v + 16 * (r >> 1) + 2 * (r & 1);
+            float acc = 0.f;
 #pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-              const float4 c = w1[h4];
-              a1 = fmaf(c.x, v[32 + 4 * h4], a1);
-              a1 = fmaf(c.y, v[32 + 4 * h4 + 1], a1);
-              a1 = fmaf(c.z, v[32 + 4 * h4 + 2], a1);
-              a1 = fmaf(c.w, v[32 + 4 * h4 + 3], a1);
+            for (int i = 0; i < 4; ++i) {
+              acc = fmaf(wr[j][2 * i], x[4 * i], acc);
+              acc = fmaf(wr[j][2 * i + 1], x[4 * i + 1], acc);
             }
+            p[r] = acc;
           }
-          sc[2 * it2] = a0;
-          sc[2 * it2 + 1] = a1;
+          // reduce-scatter over lanes t ^ 2, t ^ 1: lane t keeps key row t / 4 + 8 (t % 4)
+          const bool b1 = (lane & 2) != 0, b0 = (lane & 1) != 0;
+          float k0 = b1 ? p[2] : p[0], k1 = b1 ? p[3] : p[1];
+          const float s0 = b1 ? p[0] : p[2], s1 = b1 ? p[1] : p[3];
+          k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+          k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+          const float kk = b0 ? k1 : k0, ss = b0 ? k0 : k1;
+          sc[j] = kk + __shfl_xor_sync(0xffffffffu, ss, 1);
         }
       }
       tc_fence_before();

@@ -285,6 +285,28 @@ __device__ __forceinline__ void tmem_ld32x2_sync(uint32_t a0, uint32_t a1, float
 #pragma unroll
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
+// Two 16-lane loads of shape 16x256b, 4 repeats along the columns (32 columns each),
+// at TMEM addresses a_lo and a_hi, followed by tcgen05.wait::ld.  Thread t of the
+// warp holds, for repeat i (columns 8i .. 8i + 7 from the address):
+//   v[4i + 0], v[4i + 1]: row t / 4,     columns 8i + 2 (t % 4) + 0, + 1
+//   v[4i + 2], v[4i + 3]: row t / 4 + 8, the same columns
+// rows counted from the lane field of a_lo (v[0..15]) and of a_hi (v[16..31]).
+__device__ __forceinline__ void tmem_ld16x256b_x4x2_sync(uint32_t a_lo, uint32_t a_hi, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
+      "[%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(a_lo), "r"(a_hi)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
