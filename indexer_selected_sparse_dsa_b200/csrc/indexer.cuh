@@ -19,9 +19,12 @@
 // (one key per lane).  No weight is re-read from shared memory per key unit,
 // which leaves the shared-memory pipe to the tensor core's operand reads.
 //
-// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
-// and MMA issuer, warps 2..9 = epilogue (two warps per TMEM lane quarter, each
-// taking every other query of the tile).  Persistent grid.
+// Warp roles: warp 0 = TMA producer, warp 1 = TMEM allocator and MMA issuer,
+// warps 2.. = epilogue, P warps per TMEM lane quarter (P = 4 for the 8-query
+// tile, else 2), warp part p taking queries p, p + P, ...  Each warp works
+// through its share of a unit serially (TMEM load, head sum, store or filter),
+// so that share, not the tensor core, sets the pace unless it is small: four
+// warps per quarter keep it at two queries.  Persistent grid.
 //
 // Streamed selection (STREAM): no score is written.  Each score above its
 // query's filter threshold goes, with its position, into the query's
@@ -242,8 +245,15 @@ struct UnitIter {
 };
 
 // ------------------------------------------------------------------ main kernel
-constexpr int kEpiWarps = 8;
-constexpr int kIdxThreads = 64 + 32 * kEpiWarps;
+// Epilogue warps of a tile of QMAX queries (a multiple of 4: whole lane quarters).
+template <int QMAX>
+__host__ __device__ constexpr int epi_warps() {
+  return QMAX == 8 ? 16 : 8;
+}
+template <int QMAX>
+__host__ __device__ constexpr int idx_threads() {
+  return 64 + 32 * epi_warps<QMAX>();
+}
 constexpr int kCheckUnits = 32;  // streaming selection: units between candidate-buffer checks
 static_assert(kStreamCap - DSA_MAX_TOPK >= kCheckUnits * kKeysPerUnit,
               "a cut buffer must take every key of one check interval");
@@ -272,12 +282,15 @@ struct IdxSmem {
 };
 
 template <int QMAX, int STAGES, int QBUF, bool STREAM>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const uint16_t* __restrict__ w, const int32_t* __restrict__ n_vis,
                    const PlanHeader* __restrict__ hdr, const PlanTile* __restrict__ tiles, float* __restrict__ scores,
                    int64_t score_ld, int sweep, StreamOut so, WaitLimit lim) {
   using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
+  constexpr int EPI = epi_warps<QMAX>();  // epilogue warps
+  constexpr int P = EPI / 4;              // epilogue warps per TMEM lane quarter
+  constexpr int J = (QMAX + P - 1) / P;   // queries per epilogue warp (at most)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -307,7 +320,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(afull_bar(b), 1);
-      mbar_init(aempty_bar(b), kEpiWarps);  // one arrival per epilogue warp
+      mbar_init(aempty_bar(b), EPI);  // one arrival per epilogue warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -421,13 +434,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_wait(drain_bar, 0, lim, nullptr);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..9)
+    // ---------------------------------------------------------------- epilogue (warps 2 .. 1 + EPI)
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;     // queries half, half + 2, half + 4, ...
+    const int part = (warp - 2) >> 2;     // queries part, part + P, part + 2P, ...
     // after the head reduce-scatter lane t holds key row t / 4 + 8 (t % 4) of the quarter
     const int row = quarter * 32 + (lane >> 2) + 8 * (lane & 3);
     const int hc = 2 * (lane & 3);        // this lane's heads: 8i + hc + {0, 1}, i < 4
-    const int et = threadIdx.x - 64;      // 0 .. 32 * kEpiWarps - 1
+    const int et = threadIdx.x - 64;      // 0 .. 32 * EPI - 1
     long long* thr_s = reinterpret_cast<long long*>(smem + L::kThrOff);
     int* cnt_s = reinterpret_cast<int*>(smem + L::kCntOff);
     int* seeded_s = reinterpret_cast<int*>(smem + L::kSmpOff);
@@ -506,16 +519,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (seeded_s[q] && cnt_s[q] < min(so.topk, nv_s[q])) so.redo[1 + atomicAdd(so.redo, 1)] = q0 + q;
       else so.cnt_out[q0 + q] = min(cnt_s[q], so.cap);
     };
-    // This thread's queries are half, half + 2, half + 4, half + 6 (slot j: half + 2j);
+    // This thread's queries are part + P j, j < J (slot j);
     // their visible lengths and filter thresholds live in registers, reloaded from
     // shared memory only where they change (tile start, seeding, buffer checks).
-    int nv_r[4];
-    long long thr_r[4];
-    float wr[4][8];  // wr[j][2i + e] = w[query half + 2j, head 8i + hc + e]
+    int nv_r[J];
+    long long thr_r[J];
+    float wr[J][8];  // wr[j][2i + e] = w[query part + P j, head 8i + hc + e]
     auto refresh = [&]() {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int q = half + 2 * j;
+      for (int j = 0; j < J; ++j) {
+        const int q = part + P * j;
         nv_r[j] = q < QMAX ? nv_s[q] : 0;
         thr_r[j] = (STREAM && q < QMAX) ? thr_s[q] : -1;
       }
@@ -529,8 +542,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     while (ok) {
       const int nq = it.cur.nq;
       if (it.tile != prev_tile) {
-        named_bar_sync(1, 32 * kEpiWarps);
-        for (int e = et; e < nq * 32; e += 32 * kEpiWarps)
+        named_bar_sync(1, 32 * EPI);
+        for (int e = et; e < nq * 32; e += 32 * EPI)
           w_s[e] = bf16_bits_to_float(w[(long long)it.cur.q0 * 32 + e]);
         if (et < QMAX) nv_s[et] = et < nq ? n_vis[it.cur.q0 + et] : 0;
         if constexpr (STREAM) {
@@ -540,11 +553,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             seeded_s[et] = 0;
           }
         }
-        named_bar_sync(1, 32 * kEpiWarps);
+        named_bar_sync(1, 32 * EPI);
         refresh();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int q = half + 2 * j;
+        for (int j = 0; j < J; ++j) {
+          const int q = part + P * j;
 #pragma unroll
           for (int e = 0; e < 8; ++e) wr[j][e] = q < nq ? w_s[q * 32 + 8 * (e >> 1) + hc + (e & 1)] : 0.f;
         }
@@ -555,9 +568,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const long long s = (long long)it.unit() * kKeysPerUnit + row;
       const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
       // score of (query qi, key s): written out, or offered to the query's candidate buffer
-      // append the passing scores of query slot j (qi = half + 2j) to its buffer
+      // append the passing scores of query slot j (qi = part + P j) to its buffer
       auto append = [&](int j, uint32_t key, bool pass) {
-        const int qi = half + 2 * j;
+        const int qi = part + P * j;
         const unsigned m = __ballot_sync(0xffffffffu, pass);
         if (m) {
           const int leader = __ffs(m) - 1;
@@ -572,13 +585,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
         }
       };
-      // This warp's queries qi = half, half + 2, half + 4, half + 6, one TMEM wait each.
+      // This warp's queries qi = part + P j, one TMEM wait each.
       // All scores are computed first and the accumulator is handed back to the
       // MMA warp before any is written or offered to a selection buffer.
-      float sc[4];
+      float sc[J];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int qi = half + 2 * j;
+      for (int j = 0; j < J; ++j) {
+        const int qi = part + P * j;
         sc[j] = 0.f;
         if (qi < nq) {  // warp-uniform
           float v[32];
@@ -612,27 +625,27 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (lane == 0) mbar_arrive(aempty_bar(ab));
       if constexpr (!STREAM) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (s < nv_r[j]) scores[(long long)(it.cur.q0 + half + 2 * j) * score_ld + s] = sc[j];
+        for (int j = 0; j < J; ++j)
+          if (s < nv_r[j]) scores[(long long)(it.cur.q0 + part + P * j) * score_ld + s] = sc[j];
       } else {
         // one vote for the common case that no score of the warp passes its filter
-        uint32_t key[4];
-        bool pass[4];
+        uint32_t key[J];
+        bool pass[J];
         bool any = false;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < J; ++j) {
           key[j] = float_order_key(sc[j]);
           pass[j] = s < nv_r[j] && (long long)key[j] > thr_r[j];
           any = any || pass[j];
         }
         if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (half + 2 * j < nq) append(j, key[j], pass[j]);
+          for (int j = 0; j < J; ++j)
+            if (part + P * j < nq) append(j, key[j], pass[j]);
         }
       }
       if constexpr (STREAM) {
-        const Group g{et, 32 * kEpiWarps, 1};
+        const Group g{et, 32 * EPI, 1};
         if (it.kt < 0) {
           // the sample units fill at most kSampleUnits * 128 = cap entries; after
           // the last one, seed each query's threshold
@@ -687,7 +700,7 @@ cudaError_t launch_main(const IndexerLaunch& p, const CUtensorMap& tk, const CUt
   using L = IdxSmem<QMAX, STAGES, QBUF, STREAM>;
   auto* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   auto* tiles = reinterpret_cast<const PlanTile*>(reinterpret_cast<const uint8_t*>(p.plan) + sizeof(PlanHeader));
-  return launch_pdl(indexer_kernel<QMAX, STAGES, QBUF, STREAM>, dim3(p.grid), dim3(kIdxThreads), L::kAlloc,
+  return launch_pdl(indexer_kernel<QMAX, STAGES, QBUF, STREAM>, dim3(p.grid), dim3(idx_threads<QMAX>()), L::kAlloc,
                     p.stream, 1, tk, tq, p.w, p.n_vis, hdr, tiles, p.scores, p.score_ld, p.sweep, p.stream_out,
                     WaitLimit{p.wait_ns});
 }
