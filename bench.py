@@ -502,10 +502,16 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
     """dsa_forward with the step's inputs copied in from pinned host memory and
     its result copied out, every step.  The cache stays resident (it is state
     that persists across decode steps); the rows this step appends to it (the
-    new token's k_I and latent row of each sequence) are part of the copy-in."""
+    new token's k_I and latent row of each sequence) are part of the copy-in.
+
+    Pipelined (default): two sets of input and output buffers; step i + 1's
+    copy-in (one copy stream) and step i - 1's copy-out (another) run while
+    step i computes, as a serving loop would.  --e2e-serial runs copy-in,
+    compute and copy-out of each step back to back on one stream instead."""
     import torch
     from indexer_selected_sparse_dsa_b200 import binding as B
-    T = c.T
+    serial = args.e2e_serial
+    nb = 1 if serial else 2
     new_rows = (c.kv_start + c.n_vis.to(torch.int64) - 1)
     h = {
         "q_I": c.q_I.cpu().pin_memory(), "w": c.w.cpu().pin_memory(), "q": c.q.cpu().pin_memory(),
@@ -513,28 +519,56 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
         "k_new": c.k_I[new_rows].cpu().pin_memory(), "kv_new": c.kv[new_rows].cpu().pin_memory(),
         "rows": new_rows.cpu().pin_memory(),
     }
-    d = {kk: torch.empty_like(v, device=dev) for kk, v in h.items()}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    d = [{kk: torch.empty_like(v, device=dev) for kk, v in h.items()} for _ in range(nb)]
+    o_d = [o] + [torch.empty_like(o) for _ in range(nb - 1)]
+    lse_d = [lse] + [torch.empty_like(lse) for _ in range(nb - 1)]
+    o_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(nb)]
+    lse_h = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(nb)]
     bi = sum(v.numel() * v.element_size() for v in h.values())
-    bo = o_h.numel() * 4 + lse_h.numel() * 4
+    bo = o_h[0].numel() * 4 + lse_h[0].numel() * 4
+    cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nb)]    # buffer set b: inputs landed
+    ev_done = [torch.cuda.Event() for _ in range(nb)]  # buffer set b: step computed (inputs consumed)
+    ev_out = [torch.cuda.Event() for _ in range(nb)]   # buffer set b: outputs copied out
 
-    def step_on_stream():
-        for kk in h:
-            d[kk].copy_(h[kk], non_blocking=True)
-        c.k_I.index_copy_(0, d["rows"], d["k_new"])
-        c.kv.index_copy_(0, d["rows"], d["kv_new"])
-        B.dsa_forward(d["q_I"], d["w"], c.k_I, d["q"], c.kv, d["kv_start"], d["n_vis"], max_n, k, wl.SCALE,
-                      o, lse, idx, ws, stream)
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+    def compute(b):
+        c.k_I.index_copy_(0, d[b]["rows"], d[b]["k_new"])
+        c.kv.index_copy_(0, d[b]["rows"], d[b]["kv_new"])
+        B.dsa_forward(d[b]["q_I"], d[b]["w"], c.k_I, d[b]["q"], c.kv, d[b]["kv_start"], d[b]["n_vis"], max_n, k,
+                      wl.SCALE, o_d[b], lse_d[b], idx, ws, stream)
 
-    def step():
-        with torch.cuda.stream(stream):   # copies, cache update and dsa_forward in one stream order
-            step_on_stream()
+    def step(i):
+        b = i % nb
+        if serial:
+            with torch.cuda.stream(stream):   # copies, cache update and dsa_forward in one stream order
+                for kk in h:
+                    d[b][kk].copy_(h[kk], non_blocking=True)
+                compute(b)
+                o_h[b].copy_(o_d[b], non_blocking=True)
+                lse_h[b].copy_(lse_d[b], non_blocking=True)
+            return
+        with torch.cuda.stream(cin):
+            cin.wait_event(ev_done[b])        # the step that last used set b has read its inputs
+            for kk in h:
+                d[b][kk].copy_(h[kk], non_blocking=True)
+            ev_in[b].record(cin)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])      # set b's previous outputs have left the device
+            compute(b)
+            ev_done[b].record(stream)
+        with torch.cuda.stream(cout):
+            cout.wait_event(ev_done[b])
+            o_h[b].copy_(o_d[b], non_blocking=True)
+            lse_h[b].copy_(lse_d[b], non_blocking=True)
+            ev_out[b].record(cout)
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    def run(n):
+        for i in range(n):
+            step(i)
+        stream.wait_stream(cout)              # the last copy-out is part of the run
+
+    run(max(3, args.warmup))
     torch.cuda.synchronize(dev)
     steps = args.steps
     if dist:
@@ -542,8 +576,8 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        step()
+    cin.wait_stream(stream)                   # the first copy-in starts inside the timed region
+    run(steps)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     if dist:
@@ -551,7 +585,8 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
     ms = reduce_max_ms(e0.elapsed_time(e1), dist, dev)
     B.dsa_sync_status(stream)
     return {"ms_per_step": ms / steps, "unit": "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s",
-            "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "api": "dsa_forward"}
+            "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "api": "dsa_forward",
+            "mode": "serial" if serial else "pipelined: step i+1 copy-in and step i-1 copy-out overlap step i"}
 
 
 def cpu_baseline(c, o, lse, idx, args, budget_s: float = 15.0):
@@ -660,6 +695,8 @@ def main():
     ap.add_argument("--scale", type=int, default=1, help="shrink contexts by this factor (small captures)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--e2e-serial", action="store_true",
+                    help="end-to-end leg: copy-in, compute and copy-out of each step back to back on one stream")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time eager launches instead of replaying the step captured as a CUDA graph")
     ap.add_argument("--dense-window", type=int, default=0,
