@@ -121,6 +121,33 @@ def test_topk_bit_exact(kind, k, split, monkeypatch):
         assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
 
 
+@pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "comb", "strided"])
+@pytest.mark.parametrize("k", [7, 2048])
+@pytest.mark.parametrize("split", [None, "4"])
+def test_topk_dense_rows_exact(kind, k, split, monkeypatch):
+    # rows from just above the on-chip candidate buffer (10240 keys) to 32769
+    # keys: the sampled, streamed path with its cuts, near the 32K boundary
+    if split:
+        monkeypatch.setenv("DSA_TOPK_SPLIT", split)
+    lens = [10241, 16383, 30001, 32767, 32768, 32769]
+    ld = 32772
+    S = np.full((len(lens), ld), np.nan, np.float32)
+    for i, n in enumerate(lens):
+        if kind == "comb":      # a tie class straddling the k-th place, spread over the row
+            S[i, :n] = np.where(np.arange(n) % 5 == 0, 1.0, np.arange(n) * -1e-6).astype(np.float32)
+        elif kind == "strided":  # high scores exactly on a strided sample's positions: the sample
+            st = max(1, n // 4096)  # threshold then admits fewer than k keys (the full radix select runs)
+            r = np.random.default_rng(7 * i)
+            S[i, :n] = np.where(np.arange(n) % st == 0, 1.0 + r.random(n), np.arange(n) * -1e-6).astype(np.float32)
+        else:
+            S[i, :n] = _topk_case(kind, n, seed=31 * i + k)
+    n_vis = np.array(lens, np.int32)
+    ref = oracle.topk(S.astype(np.float64), n_vis, k)
+    got = gpu_topk(S, n_vis, k)
+    for i in range(len(lens)):
+        assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
+
+
 @pytest.mark.parametrize("path,split", [("filtered", "1"), ("filtered", "2"), ("filtered", "4"), ("full", "1"),
                                         ("full", "2")])
 def test_topk_long_rows_exact(path, split, monkeypatch):
