@@ -123,10 +123,10 @@ def test_topk_bit_exact(kind, k, split, monkeypatch):
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "comb", "strided"])
 @pytest.mark.parametrize("k", [7, 2048])
-@pytest.mark.parametrize("split", [None, "4"])
+@pytest.mark.parametrize("split", [None, "2", "4"])
 def test_topk_dense_rows_exact(kind, k, split, monkeypatch):
     # rows from just above the on-chip candidate buffer (10240 keys) to 32769
-    # keys: the sampled, streamed path with its cuts, near the 32K boundary
+    # keys, streamed by one CTA or a cluster (sampled threshold, cuts, merge)
     if split:
         monkeypatch.setenv("DSA_TOPK_SPLIT", split)
     lens = [10241, 16383, 30001, 32767, 32768, 32769]
