@@ -584,9 +584,13 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
         dist.barrier()
     ms = reduce_max_ms(e0.elapsed_time(e1), dist, dev)
     B.dsa_sync_status(stream)
+    # every step computes the same batch: each buffer set's copied-out result must
+    # equal the device-resident run's (the kernels are deterministic)
+    same = all(torch.equal(o_h[b], o_d[0].cpu()) and torch.equal(lse_h[b], lse_d[0].cpu()) for b in range(nb))
     return {"ms_per_step": ms / steps, "unit": "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s",
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "api": "dsa_forward",
-            "mode": "serial" if serial else "pipelined: step i+1 copy-in and step i-1 copy-out overlap step i"}
+            "mode": "serial" if serial else "pipelined: step i+1 copy-in and step i-1 copy-out overlap step i",
+            "outputs_match_device_run": bool(same)}
 
 
 def cpu_baseline(c, o, lse, idx, args, budget_s: float = 15.0):
