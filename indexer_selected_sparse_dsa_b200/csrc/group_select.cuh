@@ -67,14 +67,15 @@ struct Rule {
 };
 
 // Exact selection of the need-th largest key among the m entries with inc(j);
-// key(j) returns a 32-bit order key.  hist holds >= 4096 words.
+// key(j) returns a 32-bit order key.  The digits, from the top, are
+// widths[0 .. npass - 1] bits wide (summing to 32); hist holds
+// 1 << max(widths) words.
 template <class Key, class Inc>
-__device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared& gs, const Group& g, Key key,
-                                   Inc inc) {
+__device__ Rule group_radix_select_digits(int m, int need, uint32_t* hist, GroupShared& gs, const Group& g, Key key,
+                                          Inc inc, const int* widths, int npass) {
   uint32_t prefix = 0;
   int bits_done = 0;
-  const int widths[3] = {12, 10, 10};
-  for (int p = 0; p < 3; ++p) {
+  for (int p = 0; p < npass; ++p) {
     const int w = widths[p];
     const int shift = 32 - bits_done - w;
     const int nb = 1 << w;
@@ -125,9 +126,17 @@ __device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared&
     const int count = gs.sel_count;
     g.sync();
     if (count == need) return Rule{((long long)prefix << (32 - bits_done)) - 1, 0, 0};
-    if (p == 2) return Rule{(long long)prefix, need, count};
+    if (p == npass - 1) return Rule{(long long)prefix, need, count};
   }
   return Rule{0, 0, 0};  // not reached
+}
+
+// The same with 12 + 10 + 10 bit digits (three passes; hist holds 4096 words).
+template <class Key, class Inc>
+__device__ Rule group_radix_select(int m, int need, uint32_t* hist, GroupShared& gs, const Group& g, Key key,
+                                   Inc inc) {
+  const int widths[3] = {12, 10, 10};
+  return group_radix_select_digits(m, need, hist, gs, g, key, inc, widths, 3);
 }
 
 // In-place stable compaction: entry j (read with load(j)) is kept when keep(e);

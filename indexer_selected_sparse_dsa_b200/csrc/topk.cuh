@@ -38,6 +38,7 @@
 #include "dsa.h"
 #include "internal.h"
 #include "ptx.cuh"
+#include "topk_short.cuh"
 
 namespace dsa {
 
@@ -626,6 +627,8 @@ cudaError_t prepare_topk() {
   cudaError_t e =
       cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(TopkShared)));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(topk_short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(ShortShared)));
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(stream_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               int(sizeof(TopkShared)));
 }
@@ -640,8 +643,15 @@ cudaError_t launch_stream_select(const StreamOut& so, const int32_t* n_vis, int 
 cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int topk, int32_t* idx,
                         int sm_count, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
-  const char* force = std::getenv("DSA_TOPK_KERNEL");  // "row": skip the filter (tests of the full path)
+  // DSA_TOPK_KERNEL (tests): "row" skips the filter of the row kernel (its full
+  // radix path), "short" takes the short-row kernel for any batch size
+  const char* force = std::getenv("DSA_TOPK_KERNEL");
   const int force_full = (force && force[0] == 'r') ? 1 : 0;
+  const bool force_short = force && force[0] == 's';
+  // Many short rows: three 256-thread CTAs per SM, one row each.
+  if (!force_full && score_ld <= kShortMaxN && (force_short || T >= 2 * sm_count))
+    return launch_pdl(topk_short_kernel, dim3(unsigned(T)), dim3(kShortThreads), sizeof(ShortShared), stream, 1,
+                      scores, score_ld, n_vis, topk, idx);
   // Few rows: split each long row over a cluster so more SMs stream it.
   int split = 1;
   if (const char* sp = std::getenv("DSA_TOPK_SPLIT")) {  // tests pin 1, 2 or 4

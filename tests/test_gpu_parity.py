@@ -104,10 +104,13 @@ def _topk_case(kind, n, seed):
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "wide"])
 @pytest.mark.parametrize("k", [1, 7, 2048])
-@pytest.mark.parametrize("split", [None, "4"])
+@pytest.mark.parametrize("split", [None, "4", "short"])
 def test_topk_bit_exact(kind, k, split, monkeypatch):
-    # split "4": every row over a cluster of 4 CTAs (a 20000-key row leaves one idle)
-    if split:
+    # split "4": every row over a cluster of 4 CTAs (a 20000-key row leaves one idle);
+    # "short": the short-row kernel (256 threads per row, three rows per SM)
+    if split == "short":
+        monkeypatch.setenv("DSA_TOPK_KERNEL", "short")
+    elif split:
         monkeypatch.setenv("DSA_TOPK_SPLIT", split)
     lens = [1, 5, k - 1 if k > 1 else 1, k, k + 1, 2047, 2049, 5000, 20000]
     ld = (max(lens) + 3) // 4 * 4
@@ -123,14 +126,18 @@ def test_topk_bit_exact(kind, k, split, monkeypatch):
 
 @pytest.mark.parametrize("kind", ["normal", "ties", "equal", "zeros", "comb", "strided"])
 @pytest.mark.parametrize("k", [7, 2048])
-@pytest.mark.parametrize("split", [None, "2", "4"])
+@pytest.mark.parametrize("split", [None, "2", "4", "short"])
 def test_topk_dense_rows_exact(kind, k, split, monkeypatch):
     # rows from just above the on-chip candidate buffer (10240 keys) to 32769
-    # keys, streamed by one CTA or a cluster (sampled threshold, cuts, merge)
-    if split:
+    # keys, streamed by one CTA or a cluster (sampled threshold, cuts, merge);
+    # "short": up to 32768 keys through the short-row kernel, whose buffer
+    # (6144) the combs, equal rows and strided rows overflow or starve
+    if split == "short":
+        monkeypatch.setenv("DSA_TOPK_KERNEL", "short")
+    elif split:
         monkeypatch.setenv("DSA_TOPK_SPLIT", split)
-    lens = [10241, 16383, 30001, 32767, 32768, 32769]
-    ld = 32772
+    lens = [10241, 16383, 30001, 32767, 32768] + ([] if split == "short" else [32769])
+    ld = 32768 if split == "short" else 32772
     S = np.full((len(lens), ld), np.nan, np.float32)
     for i, n in enumerate(lens):
         if kind == "comb":      # a tie class straddling the k-th place, spread over the row
@@ -146,6 +153,24 @@ def test_topk_dense_rows_exact(kind, k, split, monkeypatch):
     got = gpu_topk(S, n_vis, k)
     for i in range(len(lens)):
         assert np.array_equal(got[i], ref[i]), f"{kind} k={k} row {i} n={lens[i]}"
+
+
+def test_topk_short_row_batch_exact():
+    # a prefill-like batch: enough rows (>= 2 x the SM count) of at most 32768
+    # scores that the launcher picks the short-row kernel by itself; lengths
+    # from 1 to 32768, every score kind, ties at the k-th place
+    r = np.random.default_rng(77)
+    T, ld, k = 320, 32768, 2048
+    lens = np.concatenate([[1, 2, 2047, 2048, 2049, 6143, 6144, 6145, 32768],
+                           r.integers(1, ld + 1, T - 9)]).astype(np.int32)
+    kinds = ["normal", "ties", "equal", "zeros", "wide"]
+    S = np.full((T, ld), np.nan, np.float32)
+    for i, n in enumerate(lens):
+        S[i, :n] = _topk_case(kinds[i % len(kinds)], int(n), seed=1000 + i)
+    ref = oracle.topk(S.astype(np.float64), lens, k)
+    got = gpu_topk(S, lens, k)
+    for i in range(T):
+        assert np.array_equal(got[i], ref[i]), f"row {i} n={lens[i]} kind={kinds[i % len(kinds)]}"
 
 
 @pytest.mark.parametrize("path,split", [("filtered", "1"), ("filtered", "2"), ("filtered", "4"), ("full", "1"),
