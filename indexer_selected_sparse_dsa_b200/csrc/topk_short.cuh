@@ -9,8 +9,8 @@
 // The row kernel of topk.cuh gives each row a 1024-thread CTA that fills an SM;
 // on a row of a few thousand scores its phases are short and separated by
 // block-wide barriers, so the SM mostly waits.  Here a row gets a 256-thread
-// CTA of about 70 KB, three rows share an SM and one row's barrier waits
-// overlap another's work.  Per row:
+// CTA of 41 KB and 48 registers a thread, five rows share an SM and one row's
+// barrier waits overlap another's work.  Per row:
 //   1. a row longer than the candidate buffer takes a strided sample of 1024
 //      keys and selects its rank-th largest, rank a few standard deviations
 //      above the sample's expected share of k: keys above that threshold t are
@@ -44,23 +44,24 @@ namespace {
 
 constexpr int kShortThreads = 256;
 constexpr int kShortMaxN = 32768;                       // longest row this kernel takes
-constexpr int kShortCap = 6144;                         // candidate entries
+constexpr int kShortCap = 4608;                         // candidate entries (about 4 sigma above a 32K row's expectation)
 constexpr int kShortSamples = 4 * kShortThreads;        // 1024
 constexpr int kShortBitmapWords = kShortMaxN / 32;      // one bit per position
 constexpr int kShortWordsPerThread = kShortBitmapWords / kShortThreads;
-constexpr int kShortVec = 8;                            // float4 loads in flight per thread
-constexpr int kShortSub = 4;                            // float4s filtered at a time
+constexpr int kShortVec = 2;                            // float4 loads in flight per thread
+constexpr int kShortSub = 2;                            // float4s filtered at a time
 static_assert(kShortCap >= kShortSamples, "the sample sits in the candidate keys");
 static_assert(kShortCap > DSA_MAX_TOPK, "the buffer holds more than k candidates");
 
 // Radix digits of the selections: four 8-bit passes, so each pass clears and
 // scans a 256-bin histogram (one bin per thread) instead of 4096 bins.
-__device__ constexpr int kShortDigits[4] = {8, 8, 8, 8};
+constexpr int kShortBins = 256;
+__device__ constexpr int kShortDigits[4] = {8, 8, 8, 8};  // 1 << 8 == kShortBins
 
 struct ShortShared {
   uint32_t cand_key[kShortCap];
   int32_t cand_pos[kShortCap];
-  uint32_t hist[4096];
+  uint32_t hist[kShortBins];
   uint32_t bitmap[kShortBitmapWords];
   GroupShared gs;
   int cnt;
@@ -73,7 +74,7 @@ __device__ __forceinline__ uint32_t short_order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kShortThreads, 3)
+__global__ void __launch_bounds__(kShortThreads, 5)
     topk_short_kernel(const float* __restrict__ scores, int64_t score_ld, const int32_t* __restrict__ n_vis, int topk,
                       int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t short_smem[];
