@@ -236,6 +236,19 @@ def rank_seed(cfg: int, rank: int) -> int:
 
 # ----------------------------------------------------------------------------- our arm
 
+def extra_workloads(args, world):
+    """Workloads measured after the headline one, each into the line's
+    ``workloads`` key: by default (one GPU, plain step, full size) all the
+    other four, so one run carries both halves of the metric."""
+    if args.workloads == "none":
+        return []
+    if args.workloads == "auto":
+        if world != 1 or args.scale != 1 or args.indexshare > 1 or args.dense_window > 0:
+            return []
+        return [c for c in (0, 1, 2, 3, 4) if c != args.config]
+    return [int(x) for x in args.workloads.split(",") if x.strip() and int(x) != args.config]
+
+
 def run_ours(args, rank, world, dist):
     import torch
     from indexer_selected_sparse_dsa_b200 import binding as B
@@ -245,7 +258,30 @@ def run_ours(args, rank, world, dist):
     B.lib()
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    cfg, scale = args.config, args.scale
+    out = measure(args.config, args.steps, args, dev, rank, world, dist, headline=True)
+    extras = extra_workloads(args, world)
+    if extras:
+        out["workloads"] = {}
+        for cfg in extras:
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+            r = measure(cfg, None, args, dev, rank, world, dist, headline=False)
+            out["workloads"][r["config"]["workload"]] = r
+            out["gpu_launches"] += r["gpu_launches"]
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def measure(cfg, steps, args, dev, rank, world, dist, headline):
+    """One workload: W warm-up steps, then `steps` timed steps (None: enough
+    steps for at least about one second of timed region), the per-kernel
+    breakdown, the roofline figures and, on rank 0 of a one-GPU run, the oracle
+    on a bounded sample of the same rows.  The headline workload also carries
+    the IndexShare / dense + sparse modes and the end-to-end leg."""
+    import torch
+    from indexer_selected_sparse_dsa_b200 import binding as B
+
+    scale = args.scale
     c = wl.make_workload_torch(cfg, dev, scale=scale, seed=rank_seed(cfg, rank))
     T = c.T
     n_vis_h = c.n_vis.cpu().numpy()
@@ -262,7 +298,7 @@ def run_ours(args, rank, world, dist):
     # IndexShare (N^2, section "IndexShare"): a group of L layers runs the indexer
     # and the top-k once (the full layer) and L - 1 shared layers attend over the
     # same index set with their own queries and latent caches.
-    L = max(1, args.indexshare)
+    L = max(1, args.indexshare) if headline else 1
     shared = [wl.make_shared_layer_torch(c, l, dev, seed=rank_seed(cfg, rank)) for l in range(1, L)]
     mla_ws = B.workspace(B.DSA_OP_SPARSE_MLA, T, max_n, k, device=dev)
     o_sh = [torch.empty_like(o) for _ in shared]
@@ -274,7 +310,7 @@ def run_ours(args, rank, world, dist):
     # Dense + sparse ("GLM-5.2's DSA architecture: how dense and sparse attention
     # split the work", section "DSA's core design"): the selection, then both
     # attention branches (window of W positions, selected set) fused per head.
-    W = args.dense_window
+    W = args.dense_window if headline else 0
     if W > 0:
         gate = torch.full((T, 64), 0.5, dtype=torch.float32, device=dev)   # the caller's fusion weights
         ds_ws = B.workspace(B.DSA_OP_DENSE_SPARSE, T, 0, 0, device=dev)
@@ -307,6 +343,15 @@ def run_ours(args, rank, world, dist):
     for _ in range(args.warmup):
         step()
     B.dsa_sync_status(stream)
+    if steps is None:
+        # enough steps for about a second of timed region (at least 10)
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize(dev)
+        est_ms = max((time.perf_counter() - t0) * 1e3 / 3, 1e-3)
+        steps = int(min(20000, max(10, math.ceil(1000.0 / est_ms))))
 
     # One step captured as a CUDA graph (the library's calls only enqueue kernels
     # and memsets on the stream), replayed K times: no host launch gaps.
@@ -332,7 +377,7 @@ def run_ours(args, rank, world, dist):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         ev0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             run()
         ev1.record(stream)
     torch.cuda.synchronize(dev)
@@ -356,12 +401,12 @@ def run_ours(args, rank, world, dist):
         clocks = s2.summary()
         if clocks is not None:
             clocks["note"] = "sampled during an equal-load loop right after the timed region (timed region too short)"
-    ms_step = ms / args.steps
+    ms_step = ms / steps
 
     # ---- per-kernel breakdown: the same kernels dsa_forward runs, through the component
     # entry points, with CUDA events between them on the launching stream
     streams = forward_streams(T, max_n)
-    nb = max(3, min(args.steps, 50))
+    nb = max(3, min(steps, 50))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
     wm = work_model(n_vis_h, c.kv_start.cpu().numpy())
     pk = peaks()
@@ -420,7 +465,7 @@ def run_ours(args, rank, world, dist):
     if W > 0:
         torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_t = max(3, min(args.steps, 200))
+        n_t = max(3, min(steps, 200))
         a.record(stream)
         for _ in range(n_t):
             dense_sparse()
@@ -443,7 +488,7 @@ def run_ours(args, rank, world, dist):
             b.record(stream)
             torch.cuda.synchronize(dev)
             return a.elapsed_time(b) / n
-        n_t = max(3, min(args.steps, 200))
+        n_t = max(3, min(steps, 200))
         t_full = timed(full_layer, n_t)
         q1, kv1 = shared[0]
         t_shared = timed(lambda: B.dsa_sparse_mla_attn(q1, kv1, c.kv_start, idx, wl.SCALE, o_sh[0], lse_sh[0],
@@ -457,20 +502,20 @@ def run_ours(args, rank, world, dist):
 
     # ---- end to end through dsa_forward with host buffers
     e2e = None
-    if not args.skip_e2e and plain:
+    if headline and not args.skip_e2e and plain:
         e2e = run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist)
         if e2e is not None:
             e2e["value"] = round(whole_job_rate(T, world, e2e.pop("ms_per_step")), 1)
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu and plain:
-        cpu = cpu_baseline(c, o, lse, idx, args)
+        cpu = cpu_baseline(c, o, lse, idx, cfg, budget_s=15.0 if headline else 6.0)
 
     value = whole_job_rate(T, world, ms_step)
     out = {
         "metric": metric_for(cfg), "value": round(value, 1),
         "unit": "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload, "batch_rows": T, "max_context": max_n, "topk": k,
                    "indexer_heads": 32, "indexer_dim": 128, "mla_heads": 64, "kv_lora_rank": 512, "rope_dim": 64,
@@ -483,7 +528,7 @@ def run_ours(args, rank, world, dist):
         "e2e": e2e,
         "gpu_launches": (launches_per_step(T, k, streams, torch.cuda.get_device_properties(dev).multi_processor_count)
                          + (L - 1) * attention_launches(T, k, torch.cuda.get_device_properties(dev).multi_processor_count))
-        * args.steps,
+        * steps,
         "clocks": clocks,
         "launch": graph_note or ("one CUDA graph per step (captured dsa_forward)" if args.graph else "eager launches"),
     }
@@ -493,9 +538,11 @@ def run_ours(args, rank, world, dist):
         out["dense_sparse"] = dense_info
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         # dsa_forward's kernels (its attention is the sparse branch), the dense branch, window indices, fusion
-        out["gpu_launches"] = (launches_per_step(T, k, streams, sms) + attention_launches(T, W, sms) + 2) * args.steps
-    if rank == 0:
-        print(json.dumps(out), flush=True)
+        out["gpu_launches"] = (launches_per_step(T, k, streams, sms) + attention_launches(T, W, sms) + 2) * steps
+    if not headline:
+        for key in ("n_gpus", "scaling", "vs_baseline", "data", "dtype", "e2e", "higher_is_better"):
+            out.pop(key, None)
+    return out
 
 
 def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
@@ -593,49 +640,80 @@ def run_e2e(args, c, o, lse, idx, ws, max_n, k, dev, stream, dist):
             "outputs_match_device_run": bool(same)}
 
 
-def cpu_baseline(c, o, lse, idx, args, budget_s: float = 15.0):
-    """The oracle, as it stands, on the host cores over a bounded sample of this
-    run's own query rows (their caches copied back); also reports how far the
-    GPU's outputs for those rows are from the oracle's."""
+def host_rows(c, rows):
+    """Host copies (uint16 bf16 bits) of some query rows of a device case and of
+    only their visible cache prefixes; rows of one sequence share one copy."""
     import torch
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    ks = c.kv_start[rows].cpu().numpy()
+    nv = c.n_vis[rows].cpu().numpy()
+    longest = {}
+    for s0, n in zip(ks, nv):
+        longest[int(s0)] = max(longest.get(int(s0), 0), int(n))
+    kI, kv, base, off = [], [], {}, 0
+    for s0, n in longest.items():
+        kI.append(u16(c.k_I[s0:s0 + n]))
+        kv.append(u16(c.kv[s0:s0 + n]))
+        base[s0] = off
+        off += n
+    starts = np.array([base[int(s0)] for s0 in ks], np.int64)
+    return (u16(c.q_I[rows]), u16(c.w[rows]), np.concatenate(kI), u16(c.q[rows]), np.concatenate(kv), starts,
+            nv.astype(np.int32))
+
+
+def sample_rows(T: int, n: int):
+    """n query rows spread over a batch, the last (longest) row included."""
+    if n >= T:
+        return list(range(T))
+    return sorted({int(x) for x in np.linspace(0, T - 1, n).round()})
+
+
+def cpu_baseline(c, o, lse, idx, cfg, budget_s: float = 15.0):
+    """The oracle, as it stands, on the host cores over a bounded sample of this
+    run's own query rows (their caches copied back), one row per core per
+    call; also reports how far the GPU's outputs for those rows are from the
+    oracle's."""
     import oracle
-    from indexer_selected_sparse_dsa_b200.workloads import case_to_host  # noqa: F401
     cores = os.cpu_count() or 1
     T = c.T
+    order = list(range(T)) if wl.WORKLOADS[cfg]["kind"] == "decode" else sample_rows(T, 16 * cores)
     rows_done, t_spent, maxerr = 0, 0.0, 0.0
-    order = list(range(T))
-    batch = min(cores, T)
-    while rows_done < T and t_spent < budget_s:
-        rows = order[rows_done:rows_done + batch]
-        # compact copies of just these rows' sequences
-        q_I = c.q_I[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-        w = c.w[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-        q = c.q[rows].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
-        ks = c.kv_start[rows].cpu().numpy()
-        nv = c.n_vis[rows].cpu().numpy()
-        kI_parts, kv_parts, starts = [], [], []
-        off = 0
-        for s0, n in zip(ks, nv):
-            kI_parts.append(c.k_I[int(s0):int(s0) + int(n)].view(torch.int16).cpu().numpy().view(np.uint16))
-            kv_parts.append(c.kv[int(s0):int(s0) + int(n)].view(torch.int16).cpu().numpy().view(np.uint16))
-            starts.append(off)
-            off += int(n)
-        kI = np.concatenate(kI_parts)
-        kv = np.concatenate(kv_parts)
+    while rows_done < len(order) and t_spent < budget_s:
+        rows = order[rows_done:rows_done + cores]
+        q_I, w, kI, q, kv, starts, nv = host_rows(c, rows)
         t0 = time.perf_counter()
-        o_ref, lse_ref, idx_ref = oracle.forward(q_I, w, kI, q, kv, np.array(starts, np.int64), nv, TOPK, wl.SCALE,
-                                                 nthreads=cores)
+        o_ref, lse_ref, idx_ref = oracle.forward(q_I, w, kI, q, kv, starts, nv, TOPK, wl.SCALE, nthreads=cores)
         t_spent += time.perf_counter() - t0
         rows_done += len(rows)
         g = o[rows].cpu().numpy().astype(np.float64)
         maxerr = max(maxerr, float(np.max(np.abs(g - o_ref))))
-    unit = "tokens/s" if metric_for(args.config) == METRIC_DECODE else "query-tokens/s"
+    unit = "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s"
+    what = "query rows of this run" if wl.WORKLOADS[cfg]["kind"] == "decode" else "query rows spread over this run's batch"
     return {"value": round(rows_done / t_spent, 3), "unit": unit, "cores": cores, "kind": "oracle",
-            "sample": f"{rows_done} of {T} query rows of this run (full context each), fp64 C++ oracle, {t_spent:.1f} s",
+            "sample": f"{rows_done} of {T} {what} (full causal context each, {cores} rows per call), "
+                      f"fp64 C++ oracle, {t_spent:.1f} s",
             "gpu_vs_oracle_max_abs_on_sample": maxerr}
 
 
 # ----------------------------------------------------------------------------- reference arm
+
+def reference_case(cfg: int, scale: int, rows: int):
+    """A bounded host-side sample of workload `cfg` for the oracle: `rows` query
+    rows with the workload's own context lengths.  Decode rows query one shared
+    cache of the workload's context length (the oracle's work per row is the
+    same as over a cache of its own; one cache keeps host memory bounded);
+    prefill rows are the last rows of the workload's batch (the longest
+    contexts)."""
+    seq_lens, queries, _kind = wl.workload_layout(cfg, scale)
+    if wl.WORKLOADS[cfg]["kind"] == "decode":
+        picked = [queries[j % len(queries)] for j in range(rows)]
+        L = max(n for _, n in picked)
+        return wl.make_case_numpy([L], [(0, n) for _, n in picked], seed=cfg)
+    return wl.make_case_numpy(seq_lens, queries[-rows:], seed=cfg)
+
 
 def run_reference(args, rank, world):
     if rank != 0:
@@ -643,15 +721,8 @@ def run_reference(args, rank, world):
     import oracle
     cores = os.cpu_count() or 1
     cfg, scale = args.config, args.scale
-    seq_lens, queries, _kind = wl.workload_layout(cfg, scale)
-    # a bounded host-side replica of the workload: the first few sequences / rows
-    if wl.WORKLOADS[cfg]["kind"] == "decode":
-        nseq = min(len(seq_lens), max(1, min(cores, 8)))
-        c = wl.make_case_numpy(seq_lens[:nseq], [q for q in queries if q[0] < nseq], seed=cfg)
-    else:
-        nq = min(len(queries), max(1, min(cores, 8)))
-        c = wl.make_case_numpy(seq_lens, queries[-nq:], seed=cfg)
-    rows_per_step = min(c.T, cores)
+    c = reference_case(cfg, scale, cores)
+    rows_per_step = min(c.T, cores)           # one row per core per step
     budget = 150.0
     times, rows_total = [], 0
     t_start = time.perf_counter()
@@ -674,6 +745,7 @@ def run_reference(args, rank, world):
     value = rows_total / tot
     unit = "tokens/s" if metric_for(cfg) == METRIC_DECODE else "query-tokens/s"
     workload = wl.WORKLOADS[cfg]["name"] + (f"_scale{scale}" if scale > 1 else "")
+    seq_lens, queries, _ = wl.workload_layout(cfg, scale)
     out = {"impl": "reference", "metric": metric_for(cfg), "value": round(value, 4), "unit": unit, "n_gpus": world,
            "steps": steps_done, "steps_requested": args.steps, "warmup": args.warmup,
            "ms_per_step": round(1e3 * tot / max(steps_done, 1), 2), "higher_is_better": True, "scaling": "weak",
@@ -681,8 +753,9 @@ def run_reference(args, rank, world):
            "config": {"workload": workload, "batch_rows": len(queries), "max_context": int(max(q[1] for q in queries)),
                       "topk": TOPK, "rows_per_step": rows_per_step},
            "cpu_baseline": {"kind": "oracle", "cores": cores, "value": round(value, 4), "unit": unit,
-                            "sample": f"{rows_per_step} query rows per step (full context each) of the workload, "
-                                      f"fp64 C++ oracle, {steps_done} steps in {tot:.1f} s"},
+                            "sample": f"{rows_per_step} query rows per step, one per core, with the workload's "
+                                      f"context lengths (full causal context each), fp64 C++ oracle, "
+                                      f"{steps_done} steps in {tot:.1f} s"},
            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -699,6 +772,9 @@ def main():
     ap.add_argument("--scale", type=int, default=1, help="shrink contexts by this factor (small captures)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--workloads", default="auto",
+                    help="other workloads measured after the headline into the line's 'workloads' key: "
+                         "'auto' (all others on one GPU at full size), 'none', or a comma list such as 2,4")
     ap.add_argument("--e2e-serial", action="store_true",
                     help="end-to-end leg: copy-in, compute and copy-out of each step back to back on one stream")
     ap.add_argument("--no-graph", dest="graph", action="store_false",

@@ -246,8 +246,37 @@ DSA_API int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, c
  * Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_BAD_ROW or
  * DSA_ERR_CUDA (a sticky CUDA error).
+ *
+ * The status word is one per device, not one per call or per stream: every
+ * kernel of the library on that device raises its bits in the same word.  A
+ * call on another stream that is still running may raise a bit after this
+ * one synchronised, and the first caller to read the word reports and clears
+ * the bits of every call that ran before it, whatever its stream.  Callers
+ * that drive several streams on one device should read the status at a point
+ * where the calls they want to attribute it to are the only ones that ran.
  */
 DSA_API int dsa_sync_status(dsa_stream_t stream);
+
+/*
+ * Limit, in nanoseconds, of every bounded device wait the library's kernels
+ * make (TMA, tensor-core and producer/consumer hand-offs).  A wait that runs
+ * past it gives up: its CTA stops its work, lets every copy and tensor-core
+ * operation it started finish, releases its resources and exits, and the
+ * timeout bit reported by dsa_sync_status as DSA_ERR_TIMEOUT is raised; the
+ * outputs of that call are then undefined, the CUDA context stays usable.
+ * 0 restores the default (environment variable DSA_WAIT_LIMIT_NS, else
+ * 1.5 s).  Takes effect for launches after the call; process-wide.
+ */
+DSA_API void dsa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Diagnostic of the hang protection: enqueues one CTA on `stream` that waits,
+ * under the current wait limit, on a barrier that nothing ever completes.
+ * The wait must give up; a following dsa_sync_status(stream) then returns
+ * DSA_ERR_TIMEOUT (and clears the bit).  With the default limit the probe
+ * takes 1.5 s; set a short limit first with dsa_set_wait_limit_ns.
+ */
+DSA_API int dsa_check_wait_timeout(dsa_stream_t stream);
 
 /* Message for the calling thread's last failure ("" if none). Never NULL. */
 DSA_API const char* dsa_last_error_string(void);

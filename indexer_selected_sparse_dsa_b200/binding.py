@@ -53,6 +53,10 @@ def lib():
         L.dsa_dense_sparse_attn.argtypes = [P, P, I64, P, P, P, I, I, I, P, F, P, P, P, P, SZ, P]
         L.dsa_dense_sparse_attn.restype = I
         L.dsa_indexer_scores_noalloc.restype = I
+        L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.dsa_set_wait_limit_ns.restype = None
+        L.dsa_check_wait_timeout.argtypes = [P]
+        L.dsa_check_wait_timeout.restype = I
         L.dsa_last_error_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = I
         for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_sync_status"):
@@ -213,6 +217,17 @@ def dsa_forward(q_I, w, k_I, q, kv, kv_start, n_vis, max_n_vis, topk, scale, o_l
 
 def dsa_sync_status(stream=None):
     _check(lib().dsa_sync_status(_stream(stream)))
+
+
+def dsa_set_wait_limit_ns(ns: int):
+    """Limit of every bounded device wait, in ns (0: the default)."""
+    lib().dsa_set_wait_limit_ns(int(ns))
+
+
+def dsa_check_wait_timeout(stream=None):
+    """Enqueue the hang-protection probe (a wait nothing completes); the next
+    dsa_sync_status reports DSA_ERR_TIMEOUT."""
+    _check(lib().dsa_check_wait_timeout(_stream(stream)))
 
 
 def workspace(op, T, max_n_vis, topk, device=None):

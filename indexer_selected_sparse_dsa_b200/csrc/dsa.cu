@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -90,8 +91,14 @@ int current_device(DeviceState** out) {
   return DSA_OK;
 }
 
+// Limit of every bounded device wait: dsa_set_wait_limit_ns, else the
+// environment variable DSA_WAIT_LIMIT_NS, else 1.5 s.  Read at each launch.
+std::atomic<unsigned long long> g_wait_limit_override{0};
+
 unsigned long long wait_limit_ns() {
-  static unsigned long long v = [] {
+  const unsigned long long o = g_wait_limit_override.load(std::memory_order_relaxed);
+  if (o > 0) return o;
+  static const unsigned long long v = [] {
     const char* s = std::getenv("DSA_WAIT_LIMIT_NS");
     if (s && *s) {
       unsigned long long x = std::strtoull(s, nullptr, 10);
@@ -100,6 +107,19 @@ unsigned long long wait_limit_ns() {
     return 1500000000ull;  // 1.5 s per wait
   }();
   return v;
+}
+
+// One CTA waits on an mbarrier that nothing ever completes, under the current
+// wait limit: the wait must give up and raise the timeout bit.
+__global__ void wait_probe_kernel(dsa::WaitLimit lim) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = dsa::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    dsa::mbar_init(b, 1);
+    dsa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) dsa::mbar_wait(b, 0, lim, nullptr);
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -498,18 +518,36 @@ int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, const dsa
   if (score_ld < 4 || score_ld % 4 != 0) return fail(DSA_ERR_INVALID_ARG, "score_ld must be a positive multiple of 4");
   DeviceState* dev = nullptr;
   if ((rc = current_device(&dev))) return rc;
-  if (!dev->noalloc_plan) {
+  void* plan = nullptr;
+  {
     // Once per device, with that device current: the host-side name of the array
-    // is not a device address, so ask the runtime for this device's copy.
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_plan);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(plan scratch)");
-    dev->noalloc_plan = ptr;
+    // is not a device address, so ask the runtime for this device's copy.  Under
+    // the device lock, so two threads making their first call race on nothing.
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (!dev->noalloc_plan) {
+      void* ptr = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_plan);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(plan scratch)");
+      dev->noalloc_plan = ptr;
+    }
+    plan = dev->noalloc_plan;
   }
   // The plan kernel rewrites every header and tile entry it uses, so the array
   // needs no clearing between calls.
-  return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, score_ld, dev->noalloc_plan, stream,
-                     dev->sm_count);
+  return run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, score_ld, plan, stream, dev->sm_count);
+}
+
+void dsa_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_override.store(ns, std::memory_order_relaxed); }
+
+int dsa_check_wait_timeout(dsa_stream_t stream) {
+  t_err.clear();
+  DeviceState* dev = nullptr;
+  int rc = current_device(&dev);
+  if (rc) return rc;
+  wait_probe_kernel<<<1, 32, 0, stream>>>(dsa::WaitLimit{wait_limit_ns()});
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe launch");
+  return DSA_OK;
 }
 
 int dsa_sync_status(dsa_stream_t stream) {

@@ -348,8 +348,9 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
       uint32_t phase = 0;
       uint32_t qphase[QBUF];
       for (int b = 0; b < QBUF; ++b) qphase[b] = 0;
-      int issued[STAGES];
+      int issued[STAGES], q_issued[QBUF];
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      for (int b = 0; b < QBUF; ++b) q_issued[b] = 0;
       bool ok = it.begin(hdr, tiles);
       while (ok) {
         if (it.tile != prev_tile) {
@@ -364,6 +365,7 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
             tma_load_2d(qdst + QMAX * kQBoxBytes + qi * kQBoxBytes, &tmap_q, qfull_bar(qb), 64, y);
           }
           qphase[qb] ^= 1u;
+          ++q_issued[qb];
           prev_tile = it.tile;
         }
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, lim, abort_flag)) break;
@@ -379,9 +381,12 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
         }
         ok = it.next();
       }
-      // Drain: every key stage we loaded must have landed before the CTA exits.
+      // Drain: every key stage and query buffer we loaded must have landed before
+      // the CTA exits (on an abort the MMA warp may not have consumed them).
       for (int s = 0; s < STAGES; ++s)
-        if (issued[s] > 0) mbar_wait(full_bar(s), uint32_t((issued[s] - 1) & 1), lim, nullptr);
+        if (issued[s] > 0) mbar_drain(full_bar(s), uint32_t((issued[s] - 1) & 1));
+      for (int b = 0; b < QBUF; ++b)
+        if (q_issued[b] > 0) mbar_drain(qfull_bar(b), uint32_t((q_issued[b] - 1) & 1));
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -429,9 +434,10 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
         }
         ok = it.next();
       }
-      // Drain: wait until every MMA issued above has completed.
+      // Drain: wait until every MMA issued above has completed (also after an
+      // abort: TMEM is released only once no MMA can still write it).
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, lim, nullptr);
+      mbar_drain(drain_bar, 0);
     }
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2 .. 1 + EPI)

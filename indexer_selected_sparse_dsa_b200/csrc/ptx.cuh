@@ -126,22 +126,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: returns false (and raises kStatusTimeout) when the limit passes,
-// or early when *abort (shared) is set by another role of the same CTA.
+// or early when *abort (shared) is set by another role of the same CTA.  The
+// clock and the abort flag are checked after every failed try, so even a limit
+// of a few nanoseconds gives up at the first wait that is not already complete.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WaitLimit lim,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
+  const unsigned long long t0 = globaltimer();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (abort_flag && *abort_flag) return false;
-      if (globaltimer() - t0 > lim.ns) {
-        raise_status(kStatusTimeout);
-        if (abort_flag) *abort_flag = 1;
-        return false;
-      }
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer() - t0 > lim.ns) {
+      raise_status(kStatusTimeout);
+      if (abort_flag) *abort_flag = 1;
+      return false;
     }
   }
+}
+
+// Drain before exit: copies and tensor-core operations this CTA started must be
+// complete before it releases TMEM or its shared memory.  A drain has its own
+// fixed limit, longer than any ordinary wait and independent of the caller's
+// (a short test limit must not cut a drain short); it gives up only if the
+// hardware itself stopped answering, raising kStatusTimeout.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  mbar_wait(bar, parity, WaitLimit{kDrainLimitNs}, nullptr);
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies

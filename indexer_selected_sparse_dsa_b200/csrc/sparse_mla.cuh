@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       prev_skip = cur_skip;
     }
     cp_async_wait_all();  // no copy may still be in flight when the CTA exits
+    if (pt == 0 && ntiles > 0) mbar_drain(q_full, 0);  // nor the query tile (an abort may leave it unread)
   } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && ntiles > 0) {
@@ -363,7 +364,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
       // every MMA issued above must be complete before TMEM is released
       mma_commit(drain);
-      mbar_wait(drain, 0, lim, nullptr);
+      mbar_drain(drain, 0);
     }
     __syncwarp();
   } else {

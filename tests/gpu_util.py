@@ -93,31 +93,45 @@ def assert_attention_close(o, lse, o_ref, lse_ref, rows=None):
             assert np.max(np.abs(lse[i][fin] - lse_ref[i][fin])) <= ATT_MAX_ABS, f"row {i}: lse"
 
 
-def assert_selection_ok(idx_gpu, scores_ref, n_vis, k):
+def reference_set(r, K):
+    """The oracle's kept set of one row: the unique top-K positions of the order
+    (score descending, position ascending), and the K-th score."""
+    n = r.shape[0]
+    if K >= n:
+        return np.arange(n), (np.min(r) if n else 0.0)
+    kth = np.partition(r, n - K)[n - K]          # K-th largest value
+    above = np.nonzero(r > kth)[0]
+    tied = np.nonzero(r == kth)[0]               # ascending positions: the lowest win
+    return np.sort(np.concatenate([above, tied[:K - above.size]])), kth
+
+
+def assert_selection_ok(idx_gpu, scores_ref, n_vis, k, rows=None):
     """The GPU's kept set may differ from the oracle's only at positions whose
     oracle score lies within 1e-3 * max|I| of the oracle's k-th score; and it
     must be a valid selection: ascending, -1 padded, size min(k, n_vis)."""
     for i, n in enumerate(n_vis):
+        name = i if rows is None else rows[i]
         g = idx_gpu[i]
-        K = min(k, n)
-        assert (g[K:] == -1).all(), f"row {i}: padding"
+        K = min(k, int(n))
+        assert (g[K:] == -1).all(), f"row {name}: padding"
         sel = g[:K]
-        assert (sel >= 0).all() and (sel < n).all(), f"row {i}: out of range"
-        assert (np.diff(sel) > 0).all(), f"row {i}: not strictly ascending"
+        assert (sel >= 0).all() and (sel < n).all(), f"row {name}: out of range"
+        assert (np.diff(sel) > 0).all(), f"row {name}: not strictly ascending"
         r = scores_ref[i, :n]
-        order = np.lexsort((np.arange(n), -r))
-        kth = r[order[K - 1]]
+        ref, kth = reference_set(r, K)
         band = SET_TOL_REL * np.max(np.abs(r))
-        ref_set = set(order[:K].tolist())
-        diff = ref_set.symmetric_difference(sel.tolist())
-        for s in diff:
-            assert abs(r[s] - kth) <= band, f"row {i}: position {s} differs with score gap {abs(r[s]-kth):.3e}"
+        diff = np.setxor1d(ref, sel)
+        if diff.size:
+            gap = np.abs(r[diff] - kth)
+            assert (gap <= band).all(), \
+                f"row {name}: position {int(diff[np.argmax(gap)])} differs with score gap {gap.max():.3e} > {band:.3e}"
 
 
-def host_rows(c, rows):
+def host_rows(c, rows, with_kv=True):
     """Compact host copies (uint16 bf16 bits) of some query rows of a torch case:
     their query tensors and only their own visible cache prefixes, re-based so
-    row j's sequence starts at the returned kv_start[j]."""
+    row j's sequence starts at the returned kv_start[j].  with_kv=False skips
+    the latent cache (kv is then None): enough for the indexer side."""
     import torch
 
     def u16(t):
@@ -133,10 +147,35 @@ def host_rows(c, rows):
         n = int(max(nv[q] for q in rows if int(ks[q]) == s0))
         if s0 not in seen:
             kI.append(u16(c.k_I[s0:s0 + n]))
-            kv.append(u16(c.kv[s0:s0 + n]))
+            if with_kv:
+                kv.append(u16(c.kv[s0:s0 + n]))
             seen[s0] = off
             off += n
         starts.append(seen[s0])
     return dict(q_I=u16(c.q_I[rows]), w=u16(c.w[rows]), q=u16(c.q[rows]), k_I=np.concatenate(kI),
-                kv=np.concatenate(kv), kv_start=np.array(starts, np.int64), n_vis=nv[rows].astype(np.int32),
+                kv=np.concatenate(kv) if with_kv else None, kv_start=np.array(starts, np.int64), n_vis=nv[rows].astype(np.int32),
                 plants=c.plants[rows])
+
+
+def host_selected_rows(c, rows, idx_rows):
+    """Host copies for checking the attention of some query rows: their queries
+    and only the latent-cache rows their index lists select, laid out so that
+    row j's selected rows start at kv_start[j] = j * k and its list becomes
+    0, 1, 2, ... (-1 padding kept).  The GPU's lists are ascending and unique,
+    so the oracle sees the same set in the same order."""
+    import torch
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    idx_rows = np.asarray(idx_rows, np.int32)
+    R, k = idx_rows.shape
+    dev = c.kv.device
+    ks = c.kv_start[torch.as_tensor(rows, dtype=torch.long, device=dev)]
+    it = torch.from_numpy(idx_rows).to(dev).long()
+    valid = it >= 0
+    src = torch.where(valid, ks[:, None] + it, torch.zeros_like(it))
+    kv_sel = c.kv[src.reshape(-1)].reshape(R * k, c.kv.shape[1])
+    idx_local = np.where(idx_rows >= 0, np.arange(k, dtype=np.int32)[None, :], -1).astype(np.int32)
+    return dict(q=u16(c.q[torch.as_tensor(rows, dtype=torch.long, device=dev)]), kv=u16(kv_sel),
+                kv_start=(np.arange(R, dtype=np.int64) * k), idx=idx_local)

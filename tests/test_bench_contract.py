@@ -27,6 +27,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"] == "decode_b4_ctx32k_shared"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["config"]["rows_per_step"] == cb["cores"]      # one row per host core per step
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
