@@ -544,6 +544,10 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
     it.samples = STREAM ? so.sample_units : 0;
     int prev_tile = -1, ab = 0;
     uint32_t aphase = 0;
+    // A warp whose accumulator wait fails stops working but keeps walking the
+    // same units, so it still takes every named barrier and group step the
+    // other epilogue warps take (leaving the loop early could strand them).
+    bool alive = true;
     bool ok = it.begin(hdr, tiles);
     while (ok) {
       const int nq = it.cur.nq;
@@ -569,7 +573,7 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
         }
         prev_tile = it.tile;
       }
-      if (!mbar_wait(afull_bar(ab), aphase, lim, abort_flag)) break;
+      if (alive) alive = __all_sync(0xffffffffu, mbar_wait(afull_bar(ab), aphase, lim, abort_flag));
       tc_fence_after();
       const long long s = (long long)it.unit() * kKeysPerUnit + row;
       const uint32_t tbase = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * L::kAccCols);
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
       for (int j = 0; j < J; ++j) {
         const int qi = part + P * j;
         sc[j] = 0.f;
-        if (qi < nq) {  // warp-uniform
+        if (alive && qi < nq) {  // warp-uniform
           float v[32];
           const uint32_t tq = tbase + uint32_t(qi * 32);
           tmem_ld16x256b_x4x2_sync(tq, tq + (16u << 16), v);
@@ -628,11 +632,11 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(aempty_bar(ab));
+      if (alive && lane == 0) mbar_arrive(aempty_bar(ab));
       if constexpr (!STREAM) {
 #pragma unroll
         for (int j = 0; j < J; ++j)
-          if (s < nv_r[j]) scores[(long long)(it.cur.q0 + part + P * j) * score_ld + s] = sc[j];
+          if (alive && s < nv_r[j]) scores[(long long)(it.cur.q0 + part + P * j) * score_ld + s] = sc[j];
       } else {
         // one vote for the common case that no score of the warp passes its filter
         uint32_t key[J];
@@ -641,7 +645,7 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
 #pragma unroll
         for (int j = 0; j < J; ++j) {
           key[j] = float_order_key(sc[j]);
-          pass[j] = s < nv_r[j] && (long long)key[j] > thr_r[j];
+          pass[j] = alive && s < nv_r[j] && (long long)key[j] > thr_r[j];
           any = any || pass[j];
         }
         if (__any_sync(0xffffffffu, any)) {

@@ -379,6 +379,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     float l_acc[64];
 #pragma unroll
     for (int h = 0; h < 64; ++h) l_acc[h] = 0.f;
+    // One softmax thread waits on the mbarrier; the barrier reduction then hands
+    // every softmax thread both the verdict and the memory ordering, so a failed
+    // wait ends the loop for all of them at the same point, before any named
+    // barrier inside it.
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      const bool mine = st == 0 ? mbar_wait(bar, parity, lim, abort_flag) : true;
+      return bar_red_or_128(mine ? 0 : 1) == 0;
+    };
     bool ok = true;
     for (int t = 0; t < ntiles && ok; ++t) {
       const int slot_i = (t_first + t) * kTileKeys + r;
@@ -387,7 +395,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const int s = irow[slot_i];
         valid = s >= 0 && ks + s < cache_rows;
       }
-      if (!(ok = mbar_wait(s_full(t & 1), uint32_t((t >> 1) & 1), lim, abort_flag))) break;
+      if (!(ok = wait_all(s_full(t & 1), uint32_t((t >> 1) & 1)))) break;
       tc_fence_after();
       // Lazy running max: exponents stay taken against m_use while no score of
       // the tile passes it by more than 2^kLazyRescale, which each thread checks
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
 
       // the single P buffer and O are free once the previous value product is done
-      if (t > 0 && !(ok = mbar_wait(p_free, uint32_t((t - 1) & 1), lim, abort_flag))) break;
+      if (t > 0 && !(ok = wait_all(p_free, uint32_t((t - 1) & 1)))) break;
       if (resc) {
         tc_fence_after();
         // O^T (lane = latent dim, column = head) *= alpha[head]
@@ -480,60 +488,54 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_arrive(p_full);
     }
     // the last value product must be complete before O is read
-    if (ok && ntiles > 0) mbar_wait(p_free, uint32_t((ntiles - 1) & 1), lim, abort_flag);
-    // running sums: one reduction over the tile rows
-    if (ok) {
+    if (ok && ntiles > 0) ok = wait_all(p_free, uint32_t((ntiles - 1) & 1));
+    if (ok) {  // the same in all softmax threads
+      // running sums: one reduction over the tile rows
       float r0, r1;
       reduce_scatter64<false>(l_acc, r0, r1);
       red[rw * 64 + 2 * lane] = r0;
       red[rw * 64 + 2 * lane + 1] = r1;
       named_bar_sync(1, 128);
       if (st < 64) l_run[st] = red[st] + red[64 + st] + red[128 + st] + red[192 + st];
-    }
-  }
-  // All threads: publishes l_run / m_use and makes the abort decision uniform.
-  __syncthreads();
-  if (warp >= 5 && !*abort_flag) {
-    const int st = threadIdx.x - 160;
-    const int quarter = warp & 3;
-    tc_fence_after();
-    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-    // one split: the normalised output; several: this split's unnormalised O with
-    // its running max (log2 units) and sum, merged by sparse_mla_combine_kernel
-    const bool direct = (splits == 1);
-    float* orow = direct ? o_lat + (long long)i * 64 * 512 : part + (long long)blockIdx.x * kPartFloats;
-    if (ntiles == 0) {
-      for (int e = st; e < 64 * 512; e += 128) orow[e] = 0.f;  // a split without tiles contributes nothing
-    } else {
+      named_bar_sync(1, 128);  // publishes l_run (and the last m_use) to the four warps
+      tc_fence_after();
+      // one split: the normalised output; several: this split's unnormalised O with
+      // its running max (log2 units) and sum, merged by sparse_mla_combine_kernel
+      const bool direct = (splits == 1);
+      float* orow = direct ? o_lat + (long long)i * 64 * 512 : part + (long long)blockIdx.x * kPartFloats;
+      if (ntiles == 0) {
+        for (int e = st; e < 64 * 512; e += 128) orow[e] = 0.f;  // a split without tiles contributes nothing
+      } else {
 #pragma unroll 1
-      for (int m = 0; m < 4; ++m) {
-        const int d = 128 * m + quarter * 32 + lane;
+        for (int m = 0; m < 4; ++m) {
+          const int d = 128 * m + quarter * 32 + lane;
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float o[32];
-          tmem_ld32_sync(lane_addr + kOCol + 64 * m + 32 * half, o);
+          for (int half = 0; half < 2; ++half) {
+            float o[32];
+            tmem_ld32_sync(lane_addr + kOCol + 64 * m + 32 * half, o);
 #pragma unroll
-          for (int hh = 0; hh < 32; ++hh) {
-            const int h = 32 * half + hh;
-            if (direct) {
-              const float l = l_run[h];
-              orow[h * 512 + d] = l > 0.f ? o[hh] / l : 0.f;
-            } else {
-              orow[h * 512 + d] = o[hh];
+            for (int hh = 0; hh < 32; ++hh) {
+              const int h = 32 * half + hh;
+              if (direct) {
+                const float l = l_run[h];
+                orow[h * 512 + d] = l > 0.f ? o[hh] / l : 0.f;
+              } else {
+                orow[h * 512 + d] = o[hh];
+              }
             }
           }
         }
       }
-    }
-    if (st < 64) {
-      if (direct) {
-        if (lse) {
-          const float l = l_run[st];
-          lse[(long long)i * 64 + st] = l > 0.f ? (m_use[st] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (st < 64) {
+        if (direct) {
+          if (lse) {
+            const float l = l_run[st];
+            lse[(long long)i * 64 + st] = l > 0.f ? (m_use[st] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          }
+        } else {
+          orow[64 * 512 + st] = m_use[st];
+          orow[64 * 512 + 64 + st] = l_run[st];
         }
-      } else {
-        orow[64 * 512 + st] = m_use[st];
-        orow[64 * 512 + 64 + st] = l_run[st];
       }
     }
   }
