@@ -14,6 +14,8 @@ Functions (all inputs are bf16 bit patterns as uint16 arrays):
   forward(case or arrays, topk, scale)                   -> (o_lat, lse, idx)
   dense_sparse(q, kv, kv_start, n_vis, idx, window, gate, scale)
                                                          -> (o_lat, lse_dense, lse_sparse)
+  block_sparse(q_I, w, k_I, q, kv, kv_start, n_vis, gates, scale)
+                                                         -> (o_lat, (lse x 3), branch sets)
 """
 from __future__ import annotations
 
@@ -139,3 +141,82 @@ def dense_sparse(q, kv, kv_start, n_vis, idx, window, gate, scale, nthreads=NTHR
 
 def forward_case(c, scale, nthreads=NTHREADS):
     return forward(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, c.topk, scale, nthreads)
+
+
+# ---------------------------------------------------------------------------
+# Block-level variant ("GLM-5: 744B parameters, 202K long context", section 2,
+# "Decoupled Sparse Attention"): the context is cut into 128-token blocks and
+# three branches attend, each over its own set of positions, and are fused with
+# weights: a local branch (the query's block and its neighbours, 3 x 128 = 384
+# positions, the later one masked by causality), a global anchor branch (one
+# block in every 16) and a dynamic branch (each query's 16 most relevant
+# blocks).  The page does not say how a block's relevance is scored: read here
+# as the largest lightning-indexer score among the block's visible positions,
+# the 16 best blocks kept under (score descending, block ascending).  The
+# page's fusion weights are learned; here they are the caller's gates
+# [T, 64, 3] (local, anchor, dynamic).
+# ---------------------------------------------------------------------------
+
+BLOCK = 128         # tokens per block
+BLOCK_TOPK = 16     # dynamic branch: blocks per query
+ANCHOR_EVERY = 16   # one anchor block in every 16 blocks
+LOCAL_SIDE = 1      # local branch: neighbour blocks on each side of the query's block
+
+
+def block_scores(scores, n_vis):
+    """Per row, the score of each visible block: the largest score among its
+    visible positions.  Returns a list of float arrays (one per row)."""
+    out = []
+    for i, n in enumerate(np.asarray(n_vis)):
+        n = int(n)
+        nb = (n + BLOCK - 1) // BLOCK
+        out.append(np.array([np.max(scores[i, b * BLOCK:min((b + 1) * BLOCK, n)]) for b in range(nb)]))
+    return out
+
+
+def block_branch_sets(scores, n_vis):
+    """Index lists of the three branches, ascending, -1 padded:
+    local [T, 3*128], anchor [T, ceil(max blocks / 16) * 128], dynamic [T, 16*128],
+    and the dynamic branch's blocks [T, 16]."""
+    n_vis = np.asarray(n_vis)
+    T = n_vis.shape[0]
+    max_nb = int((int(n_vis.max()) + BLOCK - 1) // BLOCK) if T else 1
+    W_loc = (2 * LOCAL_SIDE + 1) * BLOCK
+    W_anc = ((max_nb + ANCHOR_EVERY - 1) // ANCHOR_EVERY) * BLOCK
+    W_dyn = BLOCK_TOPK * BLOCK
+    loc = np.full((T, W_loc), -1, np.int32)
+    anc = np.full((T, W_anc), -1, np.int32)
+    dyn = np.full((T, W_dyn), -1, np.int32)
+    blk = np.full((T, BLOCK_TOPK), -1, np.int32)
+    bsc = block_scores(scores, n_vis)
+    for i, n in enumerate(n_vis):
+        t = int(n) - 1
+        qb = t // BLOCK
+        lo = max(0, (qb - LOCAL_SIDE) * BLOCK)
+        p = np.arange(lo, t + 1)
+        loc[i, :p.size] = p
+        p = np.concatenate([np.arange(b * BLOCK, min(b * BLOCK + BLOCK, t + 1)) for b in range(0, qb + 1, ANCHOR_EVERY)])
+        anc[i, :p.size] = p
+        order = sorted(range(qb + 1), key=lambda b: (-bsc[i][b], b))[:BLOCK_TOPK]
+        kept = sorted(order)
+        blk[i, :len(kept)] = kept
+        p = np.concatenate([np.arange(b * BLOCK, min(b * BLOCK + BLOCK, t + 1)) for b in kept])
+        dyn[i, :p.size] = p
+    return loc, anc, dyn, blk
+
+
+def block_sparse(q_I, w, k_I, q, kv, kv_start, n_vis, gates, scale, nthreads=NTHREADS):
+    """The block-level layer: indexer scores, the three branches' sets, one
+    latent attention per branch (``sparse_mla``), fused per (row, head):
+    o = sum_b gates[:, :, b] * o_b (b = local, anchor, dynamic).
+    Returns (o_lat, (lse_local, lse_anchor, lse_dynamic), sets)."""
+    S = indexer_scores(q_I, w, k_I, kv_start, n_vis, nthreads=nthreads)
+    sets = block_branch_sets(S, n_vis)
+    outs, lses = [], []
+    for idx in sets[:3]:
+        o_b, lse_b = sparse_mla(q, kv, kv_start, idx, scale, nthreads)
+        outs.append(o_b)
+        lses.append(lse_b)
+    g = np.asarray(gates, np.float64)
+    o = sum(g[:, :, b, None] * outs[b] for b in range(3))
+    return o, tuple(lses), sets

@@ -36,3 +36,39 @@ def test_pins_catch_mutant(name, tmp_path):
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+# Plausible mistakes in the block-level variant (a Python front end over the same
+# routines): each is planted in a copy of the oracle package, and the block pins
+# must fail on it.
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+BLOCK_MUTANTS = {
+    "local_two_neighbours": ("LOCAL_SIDE = 1 ", "LOCAL_SIDE = 2 "),
+    "anchor_last_block_of_16": ("for b in range(0, qb + 1, ANCHOR_EVERY)]", "for b in range(ANCHOR_EVERY - 1, qb + 1, ANCHOR_EVERY)]"),
+    "block_score_mean": ("out.append(np.array([np.max(scores[i, b * BLOCK:min((b + 1) * BLOCK, n)])",
+                         "out.append(np.array([np.mean(scores[i, b * BLOCK:min((b + 1) * BLOCK, n)])"),
+    "block_ties_to_higher": ("key=lambda b: (-bsc[i][b], b))", "key=lambda b: (-bsc[i][b], -b))"),
+    "drop_anchor_branch": ("o = sum(g[:, :, b, None] * outs[b] for b in range(3))",
+                           "o = sum(g[:, :, b, None] * outs[b] for b in (0, 2))"),
+    "dynamic_top_15": ("[:BLOCK_TOPK]", "[:BLOCK_TOPK - 1]"),
+}
+
+
+@pytest.mark.parametrize("name", ["unmutated"] + sorted(BLOCK_MUTANTS))
+def test_block_pins_catch_mutant(name, tmp_path):
+    old, new = BLOCK_MUTANTS.get(name, ("", ""))
+    src = open(PY_SRC).read()
+    assert name == "unmutated" or src.count(old) == 1, name
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text((src.replace(old, new) if old else src).replace(
+        '_HERE = os.path.dirname(os.path.abspath(__file__))', '_HERE = %r' % os.path.join(ROOT, "oracle")))
+    env = dict(os.environ, PYTHONPATH=str(tmp_path) + os.pathsep + ROOT)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "-k", "block",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=str(tmp_path), env=env, capture_output=True, text=True, timeout=600)
+    assert "passed" in r.stdout or "failed" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
+    if name == "unmutated":   # control: the copy itself passes, so a failure below is the mutation's
+        assert r.returncode == 0, r.stdout[-2000:]
+    else:
+        assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"

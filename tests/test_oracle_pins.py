@@ -355,3 +355,110 @@ def test_dense_sparse_gate_mixes_per_head():
     for i, n in enumerate(n_vis):
         ro, _ = dense_reference(q[i], kv, int(n), 1 / 16)
         assert np.max(np.abs(o_full[i] - ro)) < 1e-12
+
+
+# ------------------------------------------------------------------ block-level variant
+# ("GLM-5: 744B parameters, 202K long context", section 2: 128-token blocks, a local
+# branch over the query's block and its neighbours (O(N * 384)), an anchor block in
+# every 16, the 16 most relevant blocks per query, fused with weights)
+
+def _block_case(seed, n_vis, L=None, planted_block=None):
+    r = np.random.default_rng(seed)
+    n_vis = np.asarray(n_vis, np.int32)
+    L = int(n_vis.max()) if L is None else L
+    T = n_vis.shape[0]
+    q_I = wl.bf16_from_f32((r.standard_normal((T, 32, 128)) / np.sqrt(128)).astype(np.float32))
+    w = wl.bf16_from_f32(r.random((T, 32)).astype(np.float32))
+    k_If = (r.standard_normal((L, 128)) / np.sqrt(128)).astype(np.float32)
+    if planted_block is not None:
+        # one key aligned with row 0's mean query direction: its block must be kept
+        u = wl.bf16_to_f32(q_I[0]).mean(axis=0)
+        k_If[planted_block * oracle.BLOCK + 5] = 3.0 * u / np.linalg.norm(u)
+    k_I = wl.bf16_from_f32(k_If)
+    q = wl.bf16_from_f32(r.standard_normal((T, 64, 576)).astype(np.float32))
+    kv = wl.bf16_from_f32(r.standard_normal((L, 576)).astype(np.float32))
+    return q_I, w, k_I, q, kv, np.zeros(T, np.int64), n_vis
+
+
+def test_block_counts_match_the_pages_202k_figures():
+    g = json.load(open(os.path.join(HERE, "golden", "pages_block_counts.json")))
+    assert oracle.BLOCK == g["block_tokens"] and oracle.BLOCK_TOPK == g["dynamic_topk_blocks"]
+    n = g["context_202k_blocks"] * g["block_tokens"]             # 202752 positions
+    S = np.zeros((1, n))
+    loc, anc, dyn, blk = oracle.block_branch_sets(S, np.array([n], np.int32))
+    assert (n + oracle.BLOCK - 1) // oracle.BLOCK == g["context_202k_blocks"]
+    assert np.count_nonzero(anc[0] >= 0) == g["context_202k_anchor_blocks"] * oracle.BLOCK
+    assert loc.shape[1] == g["local_window_positions"]
+    # equal scores everywhere: the lowest 16 blocks win the ties
+    assert blk[0].tolist() == list(range(16))
+
+
+def test_block_dynamic_branch_is_dense_when_16_blocks_cover_the_context():
+    q_I, w, k_I, q, kv, ks, n_vis = _block_case(301, [1, 129, 2000, 16 * 128])
+    g = np.zeros((4, 64, 3))
+    g[:, :, 2] = 1.0
+    o, lses, sets = oracle.block_sparse(q_I, w, k_I, q, kv, ks, n_vis, g, 1 / 16)
+    for i, n in enumerate(n_vis):
+        ro, rl = dense_reference(q[i], kv, int(n), 1 / 16)
+        assert np.max(np.abs(o[i] - ro)) < 1e-12
+        assert np.max(np.abs(lses[2][i] - rl)) < 1e-12
+
+
+def test_block_local_branch_is_a_sliding_window():
+    # the query's block up to itself plus the previous block: a window of
+    # (t mod 128) + 1 + 128 positions (fewer at the start)
+    q_I, w, k_I, q, kv, ks, n_vis = _block_case(302, [1, 100, 128, 129, 383, 1000, 4097])
+    g = np.zeros((7, 64, 3))
+    g[:, :, 0] = 1.0
+    o, lses, _ = oracle.block_sparse(q_I, w, k_I, q, kv, ks, n_vis, g, 1 / 16)
+    for i, n in enumerate(n_vis):
+        t = int(n) - 1
+        W = min(int(n), t % 128 + 1 + 128)
+        ro, rl = _window_reference(q[i], kv, 0, int(n), W, 1 / 16)
+        assert np.max(np.abs(o[i] - ro)) < 1e-12
+        assert np.max(np.abs(lses[0][i] - rl)) < 1e-12
+
+
+def test_block_anchor_branch_attends_the_first_block_of_every_16():
+    q_I, w, k_I, q, kv, ks, n_vis = _block_case(303, [5000, 2049, 100])
+    g = np.zeros((3, 64, 3))
+    g[:, :, 1] = 1.0
+    o, lses, sets = oracle.block_sparse(q_I, w, k_I, q, kv, ks, n_vis, g, 1 / 16)
+    anc = sets[1]
+    # t = 4999 is in block 39: anchors 0, 16, 32 -> 384 positions; t = 2048: anchors 0, 16
+    # (block 16 holds only position 2048 so far); t = 99: block 0 up to 99
+    assert np.count_nonzero(anc[0] >= 0) == 384 and np.count_nonzero(anc[1] >= 0) == 129
+    assert np.count_nonzero(anc[2] >= 0) == 100
+    K = f32(kv)
+    for i, n in enumerate(n_vis):
+        p = np.array([s for s in range(int(n)) if (s // 128) % 16 == 0])
+        S = (f32(q[i]) @ K[p].T) / 16
+        assert np.max(np.abs(o[i] - softmax(S, axis=1) @ K[p, :512])) < 1e-12
+        assert np.max(np.abs(lses[1][i] - logsumexp(S, axis=1))) < 1e-12
+
+
+def test_block_dynamic_selection_by_brute_force_and_planted_block():
+    q_I, w, k_I, q, kv, ks, n_vis = _block_case(304, [6000, 6000, 3333], planted_block=41)
+    S = oracle.indexer_scores(q_I, w, k_I, ks, n_vis)
+    _, _, dyn, blk = oracle.block_branch_sets(S, n_vis)
+    for i, n in enumerate(n_vis):
+        n = int(n)
+        nb = (n + 127) // 128
+        best = [max(S[i, s] for s in range(b * 128, min(n, b * 128 + 128))) for b in range(nb)]
+        want = sorted(sorted(range(nb), key=lambda b: (-best[b], b))[:16])
+        assert blk[i].tolist() == want
+        pos = [s for b in want for s in range(b * 128, min(n, b * 128 + 128))]
+        assert dyn[i][:len(pos)].tolist() == pos and (dyn[i][len(pos):] == -1).all()
+    assert 41 in blk[0].tolist()                                   # the planted key's block
+
+
+def test_block_fusion_is_the_gated_sum_of_the_branches():
+    q_I, w, k_I, q, kv, ks, n_vis = _block_case(305, [3000, 700])
+    r = np.random.default_rng(306)
+    g = r.uniform(0, 1, (2, 64, 3))
+    o, _, sets = oracle.block_sparse(q_I, w, k_I, q, kv, ks, n_vis, g, 1 / 16)
+    parts = [oracle.sparse_mla(q, kv, ks, idx, 1 / 16)[0] for idx in sets[:3]]
+    for i in range(2):
+        for h in (0, 31, 63):
+            want = sum(g[i, h, b] * parts[b][i, h] for b in range(3))
+            assert np.max(np.abs(o[i, h] - want)) < 1e-12
