@@ -243,7 +243,7 @@ def extra_workloads(args, world):
     if args.workloads == "none":
         return []
     if args.workloads == "auto":
-        if world != 1 or args.scale != 1 or args.indexshare > 1 or args.dense_window > 0:
+        if world != 1 or args.scale != 1 or args.indexshare > 1 or args.dense_window > 0 or args.block_sparse:
             return []
         return [c for c in (0, 1, 2, 3, 4) if c != args.config]
     return [int(x) for x in args.workloads.split(",") if x.strip() and int(x) != args.config]
@@ -310,6 +310,16 @@ def measure(cfg, steps, args, dev, rank, world, dist, headline):
     # Dense + sparse ("GLM-5.2's DSA architecture: how dense and sparse attention
     # split the work", section "DSA's core design"): the selection, then both
     # attention branches (window of W positions, selected set) fused per head.
+    # Block-level variant ("GLM-5: 744B parameters, 202K long context", section 2):
+    # local, anchor and top-16-block branches over 128-token blocks, fused per head.
+    BS = args.block_sparse and headline
+    if BS:
+        gates_b = torch.full((T, 64, 3), 1.0 / 3.0, dtype=torch.float32, device=dev)  # the caller's weights
+        ws_b = B.workspace(B.DSA_OP_BLOCK_SPARSE, T, max_n, 0, device=dev)
+
+        def block_layer():
+            B.dsa_block_sparse_attn(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, max_n, gates_b, wl.SCALE, o,
+                                    None, None, ws_b, stream)
     W = args.dense_window if headline else 0
     if W > 0:
         gate = torch.full((T, 64), 0.5, dtype=torch.float32, device=dev)   # the caller's fusion weights
@@ -332,6 +342,9 @@ def measure(cfg, steps, args, dev, rank, world, dist, headline):
                                     stream)
 
     def step():
+        if BS:
+            block_layer()
+            return
         if W > 0:
             select()
             dense_sparse()
@@ -460,7 +473,15 @@ def measure(cfg, steps, args, dev, rank, world, dist, headline):
                     "frac": v["frac"]} for kk, v in per_kernel.items()}
     step_rf = roofline_of("dsa_forward step", ms_step, wm["step_bytes"], wm["step_flops"], pk)
 
-    plain = (L == 1 and W == 0)
+    plain = (L == 1 and W == 0 and not BS)
+    block_info = None
+    if BS:
+        nb = (max_n + 127) // 128
+        block_info = {"block_tokens": 128, "dynamic_blocks": 16, "anchor_every_blocks": 16,
+                      "local_positions": 384, "anchor_positions_max": ((nb + 15) // 16) * 128,
+                      "gates": "1/3 per branch for every (row, head)", "block_layer_ms": round(ms_step, 4),
+                      "token_step_breakdown": "the kernels and roofline of this line are the token-level step's"}
+        workload += "_blocksparse"
     dense_info = None
     if W > 0:
         torch.cuda.synchronize(dev)
@@ -530,10 +551,17 @@ def measure(cfg, steps, args, dev, rank, world, dist, headline):
                          + (L - 1) * attention_launches(T, k, torch.cuda.get_device_properties(dev).multi_processor_count))
         * steps,
         "clocks": clocks,
-        "launch": graph_note or ("one CUDA graph per step (captured dsa_forward)" if args.graph else "eager launches"),
+        "launch": graph_note or (f"one CUDA graph per step (captured {'dsa_block_sparse_attn' if BS else 'dsa_forward'})"
+                                 if args.graph else "eager launches"),
     }
     if indexshare is not None:
         out["indexshare"] = indexshare
+    if block_info is not None:
+        out["block_sparse"] = block_info
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        # plan, indexer, block scores, block top-k, index lists, 3 x attention (+ merges), fusion
+        out["gpu_launches"] = (2 + 1 + 1 + 1 + attention_launches(T, 384, sms) + attention_launches(T, 2048, sms)
+                               + attention_launches(T, block_info["anchor_positions_max"], sms) + 1) * steps
     if dense_info is not None:
         out["dense_sparse"] = dense_info
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -782,6 +810,9 @@ def main():
     ap.add_argument("--dense-window", type=int, default=0,
                     help="time the dense + sparse layer instead: selection, then attention over the selected set "
                          "and over a window of W positions, fused per head (default 0: off)")
+    ap.add_argument("--block-sparse", action="store_true",
+                    help="time the block-level variant instead: 128-token blocks, local / anchor / top-16-block "
+                         "branches fused per head (dsa_block_sparse_attn)")
     ap.add_argument("--indexshare", type=int, default=1,
                     help="layers per IndexShare group: one step = one full layer (indexer, top-k, attention) "
                          "+ L-1 layers attending over its index set (default 1: no sharing)")

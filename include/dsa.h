@@ -80,7 +80,8 @@ enum dsa_op {
   DSA_OP_SPARSE_MLA = 2,
   DSA_OP_FORWARD = 3,
   DSA_OP_INDEXER_TOPK = 4,
-  DSA_OP_DENSE_SPARSE = 5
+  DSA_OP_DENSE_SPARSE = 5,
+  DSA_OP_BLOCK_SPARSE = 6
 };
 
 /*
@@ -180,6 +181,37 @@ DSA_API int dsa_dense_sparse_attn(const dsa_bf16* q, const dsa_bf16* kv, int64_t
                                   const int64_t* kv_start, const int32_t* n_vis, const int32_t* idx, int T, int topk,
                                   int window, const float* gate, float scale, float* o_lat, float* lse_dense,
                                   float* lse_sparse, void* ws, size_t ws_bytes, dsa_stream_t stream);
+
+/*
+ * Block-level variant ("GLM-5: 744B parameters, 202K long context", section 2,
+ * "Decoupled Sparse Attention"): the context is cut into 128-token blocks and
+ * three branches attend, each over its own positions, fused with weights:
+ *  - local:   the query's block and its neighbours (3 x 128 = 384 positions; the
+ *             later neighbour is in the future): positions max(0, 128 (qb - 1)) .. t,
+ *             qb = t / 128 the query's block, t = n_vis[i] - 1;
+ *  - anchor:  one block in every 16: the visible positions of blocks 0, 16, 32, ... <= qb;
+ *  - dynamic: the query's 16 most relevant blocks.  The page does not say how a
+ *             block is scored; here its score is the largest lightning-indexer
+ *             score (dsa_indexer_scores) among its visible positions, and the 16
+ *             best blocks are kept under (score descending, block ascending).
+ * Each branch is the attention of dsa_sparse_mla_attn over its positions; the
+ * page's fusion weights are learned and here come from the caller:
+ *     o_lat[i,h,:] = gates[i,h,0] o_local + gates[i,h,1] o_anchor + gates[i,h,2] o_dynamic
+ *
+ *  q_I, w, k_I, q, kv, cache_rows, kv_start, n_vis, scale   as for dsa_forward
+ *  max_n_vis   host-side bound of n_vis (rows above it: status bit, empty branches)
+ *  gates       [T,64,3] fp32 (device)
+ *  o_lat       [T,64,512] fp32
+ *  lse         [3,T,64] fp32 (each branch's log-sum-exp: local, anchor, dynamic) or NULL
+ *  blocks_out  [T,16] int32: the dynamic branch's blocks, ascending, -1 padded; or NULL
+ *  ws          >= dsa_workspace_size(DSA_OP_BLOCK_SPARSE, T, max_n_vis, 0) bytes, 256-byte
+ *              aligned; it holds the T x max_n_vis score matrix (4 bytes per entry)
+ */
+DSA_API int dsa_block_sparse_attn(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q,
+                                  const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start,
+                                  const int32_t* n_vis, int T, int64_t max_n_vis, const float* gates, float scale,
+                                  float* o_lat, float* lse, int32_t* blocks_out, void* ws, size_t ws_bytes,
+                                  dsa_stream_t stream);
 
 /*
  * Indexer and top-k fused, without a score matrix ("2026 LLM architecture

@@ -15,7 +15,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT, DSA_ERR_UNSUPPORTED, DSA_ERR_BAD_ROW = range(7)
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD, DSA_OP_INDEXER_TOPK, DSA_OP_DENSE_SPARSE = range(6)
+(DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_SPARSE_MLA, DSA_OP_FORWARD, DSA_OP_INDEXER_TOPK, DSA_OP_DENSE_SPARSE,
+ DSA_OP_BLOCK_SPARSE) = range(7)
+BLOCK_TOPK = 16
 INDEX_HEADS, INDEX_DIM, HEADS, LATENT, ROPE, ROW, MAX_TOPK = 32, 128, 64, 512, 64, 576, 2048
 NOALLOC_MAX_ROWS = 8192
 
@@ -53,6 +55,8 @@ def lib():
         L.dsa_dense_sparse_attn.argtypes = [P, P, I64, P, P, P, I, I, I, P, F, P, P, P, P, SZ, P]
         L.dsa_dense_sparse_attn.restype = I
         L.dsa_indexer_scores_noalloc.restype = I
+        L.dsa_block_sparse_attn.argtypes = [P, P, P, P, P, I64, P, P, I, I64, P, F, P, P, P, P, SZ, P]
+        L.dsa_block_sparse_attn.restype = I
         L.dsa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.dsa_set_wait_limit_ns.restype = None
         L.dsa_check_wait_timeout.argtypes = [P]
@@ -213,6 +217,32 @@ def dsa_forward(q_I, w, k_I, q, kv, kv_start, n_vis, max_n_vis, topk, scale, o_l
     _check(lib().dsa_forward(_ptr(q_I), _ptr(w), _ptr(k_I), _ptr(q), _ptr(kv), kv.shape[0], _ptr(kv_start),
                              _ptr(n_vis), T, int(max_n_vis), topk, float(scale), _ptr(o_lat), _ptr(lse),
                              _ptr(idx_out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def dsa_block_sparse_attn(q_I, w, k_I, q, kv, kv_start, n_vis, max_n_vis, gates, scale, o_lat, lse, blocks_out, ws,
+                          stream=None):
+    """Block-level variant: local / anchor / top-16-block branches fused with
+    gates [T, 64, 3]; lse [3, T, 64] and blocks_out [T, 16] may be None."""
+    import torch
+    T = n_vis.shape[0]
+    for t_, nm in ((q_I, "q_I"), (w, "w"), (k_I, "k_I"), (q, "q"), (kv, "kv")):
+        _need(t_, torch.bfloat16, None, nm)
+    _need(q_I, torch.bfloat16, (T, INDEX_HEADS, INDEX_DIM), "q_I")
+    _need(q, torch.bfloat16, (T, HEADS, ROW), "q")
+    _need(kv, torch.bfloat16, (kv.shape[0], ROW), "kv")
+    _need(k_I, torch.bfloat16, (kv.shape[0], INDEX_DIM), "k_I")
+    _need(kv_start, torch.int64, (T,), "kv_start")
+    _need(n_vis, torch.int32, (T,), "n_vis")
+    _need(gates, torch.float32, (T, HEADS, 3), "gates")
+    _need(o_lat, torch.float32, (T, HEADS, LATENT), "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, (3, T, HEADS), "lse")
+    if blocks_out is not None:
+        _need(blocks_out, torch.int32, (T, BLOCK_TOPK), "blocks_out")
+    _need(ws, torch.uint8, None, "ws")
+    _check(lib().dsa_block_sparse_attn(_ptr(q_I), _ptr(w), _ptr(k_I), _ptr(q), _ptr(kv), kv.shape[0], _ptr(kv_start),
+                                       _ptr(n_vis), T, int(max_n_vis), _ptr(gates), float(scale), _ptr(o_lat),
+                                       _ptr(lse), _ptr(blocks_out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def dsa_sync_status(stream=None):

@@ -16,6 +16,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+#include "block_sparse.cuh"
 #include "dense_sparse.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
@@ -210,6 +211,47 @@ size_t ws_dense_sparse(int T) {
          ws_mla(T, DSA_MAX_TOPK);
 }
 
+// block-level variant: the indexer plan, the score matrix, block scores and counts,
+// the dynamic blocks, the three index lists, the local and anchor outputs, the
+// attention partials
+struct BlockLayout {
+  int64_t ld, bld;
+  int wa;
+  size_t off_scores, off_bscore, off_nblocks, off_blocks, off_loc, off_anc, off_dyn, off_oloc, off_oanc, off_part,
+      part_bytes, total;
+};
+BlockLayout block_layout(int T, int64_t max_n_vis) {
+  BlockLayout L{};
+  L.ld = score_ld_for(max_n_vis);
+  const int64_t nb = (max_n_vis + dsa::kBlockTokens - 1) / dsa::kBlockTokens;
+  L.bld = (nb + 3) / 4 * 4;
+  L.wa = int((nb + dsa::kAnchorEvery - 1) / dsa::kAnchorEvery) * dsa::kBlockTokens;
+  const size_t t = size_t(T);
+  size_t o = ws_indexer(T);
+  L.off_scores = o;
+  o += align_up(t * size_t(L.ld) * 4, 256);
+  L.off_bscore = o;
+  o += align_up(t * size_t(L.bld) * 4, 256);
+  L.off_nblocks = o;
+  o += align_up(t * 4, 256);
+  L.off_blocks = o;
+  o += align_up(t * dsa::kBlockTopk * 4, 256);
+  L.off_loc = o;
+  o += align_up(t * dsa::kLocalWidth * 4, 256);
+  L.off_anc = o;
+  o += align_up(t * size_t(L.wa) * 4, 256);
+  L.off_dyn = o;
+  o += align_up(t * dsa::kDynWidth * 4, 256);
+  L.off_oloc = o;
+  o += align_up(t * DSA_HEADS * DSA_LATENT * 4, 256);
+  L.off_oanc = o;
+  o += align_up(t * DSA_HEADS * DSA_LATENT * 4, 256);
+  L.off_part = o;
+  L.part_bytes = ws_mla(T, L.wa > dsa::kDynWidth ? L.wa : dsa::kDynWidth);
+  L.total = o + L.part_bytes;
+  return L;
+}
+
 int pick_qmax(int T) {
   const char* s = std::getenv("DSA_INDEXER_QMAX");
   if (s && *s) {
@@ -311,6 +353,7 @@ size_t dsa_workspace_size(int op, int T, int64_t max_n_vis, int topk) {
     case DSA_OP_FORWARD: return ws_forward(T, max_n_vis, topk);
     case DSA_OP_INDEXER_TOPK: return ws_indexer(T) + ws_select(T);
     case DSA_OP_DENSE_SPARSE: return ws_dense_sparse(T);
+    case DSA_OP_BLOCK_SPARSE: return max_n_vis > 0 ? block_layout(T, max_n_vis).total : 0;
     default: return 0;
   }
 }
@@ -500,6 +543,63 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   dsa::MlaLaunch p{q,    kv,  cache_rows,        kv_start,      idx,           T,     topk, scale,
                    o_lat, lse, part,              ws_mla(T, topk), dev->sm_count, wait_limit_ns(), stream};
   return run_sparse_mla(p);
+}
+
+int dsa_block_sparse_attn(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, const dsa_bf16* q,
+                          const dsa_bf16* kv, int64_t cache_rows, const int64_t* kv_start, const int32_t* n_vis, int T,
+                          int64_t max_n_vis, const float* gates, float scale, float* o_lat, float* lse,
+                          int32_t* blocks_out, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  t_err.clear();
+  int rc = check_common_rows(T, cache_rows, kv_start);
+  if (rc) return rc;
+  if (T == 0) return DSA_OK;
+  if (max_n_vis < 1 || max_n_vis > cache_rows)
+    return fail(DSA_ERR_INVALID_ARG, "max_n_vis must lie in [1, cache_rows]");
+  if (!q_I || !w || !k_I || !q || !kv || !n_vis || !gates || !o_lat || !ws)
+    return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned(q_I, 16) || !aligned(w, 16) || !aligned(k_I, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
+      !aligned(o_lat, 16) || !aligned(n_vis, 4) || !aligned(gates, 4) || !aligned(lse, 4) || !aligned(blocks_out, 4))
+    return fail(DSA_ERR_INVALID_ARG, "tensor pointers misaligned (bf16/o_lat 16 B, n_vis/gates/lse/blocks 4 B)");
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "scale must be positive and finite");
+  if (int64_t(T) * DSA_HEADS > INT32_MAX) return fail(DSA_ERR_INVALID_ARG, "T too large");
+  const BlockLayout L = block_layout(T, max_n_vis);
+  if (ws_bytes < L.total) return fail(DSA_ERR_WORKSPACE, "workspace %zu < required %zu bytes", ws_bytes, L.total);
+  DeviceState* dev = nullptr;
+  if ((rc = current_device(&dev))) return rc;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* scores = reinterpret_cast<float*>(base + L.off_scores);
+  float* bscore = reinterpret_cast<float*>(base + L.off_bscore);
+  int32_t* nblocks = reinterpret_cast<int32_t*>(base + L.off_nblocks);
+  int32_t* blocks = blocks_out ? blocks_out : reinterpret_cast<int32_t*>(base + L.off_blocks);
+  int32_t* idx_loc = reinterpret_cast<int32_t*>(base + L.off_loc);
+  int32_t* idx_anc = reinterpret_cast<int32_t*>(base + L.off_anc);
+  int32_t* idx_dyn = reinterpret_cast<int32_t*>(base + L.off_dyn);
+  float* o_loc = reinterpret_cast<float*>(base + L.off_oloc);
+  float* o_anc = reinterpret_cast<float*>(base + L.off_oanc);
+  float* part = reinterpret_cast<float*>(base + L.off_part);
+  if ((rc = run_indexer(q_I, w, k_I, cache_rows, kv_start, n_vis, T, scores, L.ld, base, stream, dev->sm_count)))
+    return rc;
+  cudaError_t e = dsa::launch_block_max(scores, L.ld, n_vis, T, int(L.bld), bscore, nblocks, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block score launch");
+  // the 16 best blocks of each row: the exact top-k over block scores (ties to the lower block)
+  if ((e = dsa::launch_topk(bscore, L.bld, nblocks, T, dsa::kBlockTopk, blocks, dev->sm_count, stream)) != cudaSuccess)
+    return cuda_fail(e, "block top-k launch");
+  if ((e = dsa::launch_block_expand(blocks, n_vis, T, L.wa, idx_loc, idx_anc, idx_dyn, stream)) != cudaSuccess)
+    return cuda_fail(e, "block index launch");
+  const size_t tl = size_t(T) * DSA_HEADS;
+  dsa::MlaLaunch pl{q,     kv,  cache_rows, kv_start,     idx_loc,       T,     dsa::kLocalWidth, scale,
+                    o_loc, lse, part,       L.part_bytes, dev->sm_count, wait_limit_ns(), stream};
+  if ((rc = run_sparse_mla(pl))) return rc;
+  dsa::MlaLaunch pa{q,     kv,  cache_rows, kv_start, idx_anc, T, L.wa, scale, o_anc, lse ? lse + tl : nullptr, part,
+                    L.part_bytes, dev->sm_count, wait_limit_ns(), stream};
+  if ((rc = run_sparse_mla(pa))) return rc;
+  dsa::MlaLaunch pd{q,     kv,  cache_rows, kv_start, idx_dyn, T, dsa::kDynWidth, scale, o_lat,
+                    lse ? lse + 2 * tl : nullptr, part, L.part_bytes, dev->sm_count, wait_limit_ns(), stream};
+  if ((rc = run_sparse_mla(pd))) return rc;
+  if ((e = dsa::launch_fuse3(o_lat, o_loc, o_anc, gates, T, dev->sm_count, stream)) != cudaSuccess)
+    return cuda_fail(e, "fusion launch");
+  return DSA_OK;
 }
 
 int dsa_indexer_scores_noalloc(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, int64_t cache_rows,

@@ -109,6 +109,19 @@ cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q);
 cudaError_t launch_window_idx(const int32_t* n_vis, int T, int window, int32_t* idx_w, cudaStream_t stream);
 cudaError_t launch_fuse(float* o, const float* o_dense, const float* gate, int T, int sm_count, cudaStream_t stream);
 
+// ------------------------------------------------------------------ block-level variant
+constexpr int kBlockTokens = 128;                     // tokens per block
+constexpr int kBlockTopk = 16;                        // dynamic branch: blocks per query
+constexpr int kAnchorEvery = 16;                      // one anchor block in every 16
+constexpr int kLocalWidth = 3 * kBlockTokens;         // local branch list: the query's block and its neighbours
+constexpr int kDynWidth = kBlockTopk * kBlockTokens;  // dynamic branch list
+cudaError_t launch_block_max(const float* scores, int64_t score_ld, const int32_t* n_vis, int T, int bld,
+                             float* bscore, int32_t* nblocks, cudaStream_t stream);
+cudaError_t launch_block_expand(const int32_t* blocks, const int32_t* n_vis, int T, int wa, int32_t* idx_loc,
+                                int32_t* idx_anc, int32_t* idx_dyn, cudaStream_t stream);
+cudaError_t launch_fuse3(float* o, const float* o_loc, const float* o_anc, const float* gates, int T, int sm_count,
+                         cudaStream_t stream);
+
 // Shared-memory opt-in sizes, set once per device.
 cudaError_t prepare_indexer();
 cudaError_t prepare_sparse_mla();

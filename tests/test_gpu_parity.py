@@ -14,8 +14,8 @@ import oracle
 from indexer_selected_sparse_dsa_b200 import binding as B
 from indexer_selected_sparse_dsa_b200 import workloads as wl
 
-from gpu_util import (SCALE, assert_attention_close, assert_scores_close, assert_selection_ok, gpu_attention,
-                      gpu_forward, gpu_scores, gpu_topk, to_dev)
+from gpu_util import (ATT_MAX_ABS, ATT_REL_L2, SCALE, SET_TOL_REL, assert_attention_close, assert_scores_close,
+                      assert_selection_ok, gpu_attention, gpu_forward, gpu_scores, gpu_topk, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -508,3 +508,67 @@ def _check_indexer_topk(c):
                        B.workspace(B.DSA_OP_INDEXER_TOPK, T, maxn, k))
     B.dsa_sync_status()
     assert np.array_equal(idx_a.cpu().numpy(), idx_b.cpu().numpy())
+
+
+# ------------------------------------------------------------------ block-level variant
+
+@pytest.mark.parametrize("seed", [61, 62])
+def test_block_sparse_matches_oracle(seed):
+    """dsa_block_sparse_attn: the dynamic blocks equal the oracle's selection on the
+    GPU's own fp32 scores (the float decision taken in one precision) and differ
+    from the fp64 oracle's only inside the tie band; the fused output and each
+    branch's lse match the oracle run on the GPU's blocks."""
+    import torch
+    lens = [20000, 7000]
+    queries = [(0, 1), (0, 100), (0, 129), (0, 2049), (0, 5000), (0, 20000), (1, 7000), (1, 3000)]
+    c = wl.make_case_numpy(lens, queries, seed=seed, n_plant=16)
+    d = to_dev(c)
+    T = c.T
+    max_n = int(c.n_vis.max())
+    r = np.random.default_rng(seed)
+    gates = r.uniform(0, 1, (T, 64, 3)).astype(np.float32)
+    o = torch.full((T, 64, 512), float("nan"), device="cuda")
+    lse = torch.full((3, T, 64), float("nan"), device="cuda")
+    blocks = torch.full((T, B.BLOCK_TOPK), -7, dtype=torch.int32, device="cuda")
+    ws = B.workspace(B.DSA_OP_BLOCK_SPARSE, T, max_n, 0)
+    B.dsa_block_sparse_attn(d["q_I"], d["w"], d["k_I"], d["q"], d["kv"], d["kv_start"], d["n_vis"], max_n,
+                            torch.from_numpy(gates).cuda(), SCALE, o, lse, blocks, ws)
+    B.dsa_sync_status()
+    ld = (max_n + 3) // 4 * 4
+    off = B.dsa_workspace_size(B.DSA_OP_INDEXER, T, max_n, 0)
+    S_gpu = ws[off:off + T * ld * 4].view(torch.float32).view(T, ld).cpu().numpy().astype(np.float64)
+    sets = oracle.block_branch_sets(S_gpu, c.n_vis)
+    g_blocks = blocks.cpu().numpy()
+    np.testing.assert_array_equal(g_blocks, sets[3])
+    # against the fp64 oracle: only swaps of blocks whose scores tie within the band
+    S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis)
+    assert_scores_close(S_gpu[:, :max_n], S_ref, c.n_vis)
+    bs = oracle.block_scores(S_ref, c.n_vis)
+    _, _, _, ref_blocks = oracle.block_branch_sets(S_ref, c.n_vis)
+    for i in range(T):
+        diff = set(ref_blocks[i][ref_blocks[i] >= 0].tolist()) ^ set(g_blocks[i][g_blocks[i] >= 0].tolist())
+        if diff:
+            kth = np.sort(bs[i])[::-1][15]
+            band = SET_TOL_REL * np.max(np.abs(S_ref[i, :c.n_vis[i]]))
+            assert all(abs(bs[i][b] - kth) <= band for b in diff), f"row {i}: blocks {diff}"
+    # attention: the oracle on the GPU's branch sets, fused with the same gates
+    outs, lses = [], []
+    for idx in sets[:3]:
+        ob, lb = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+        outs.append(ob)
+        lses.append(lb)
+    o_ref = sum(gates.astype(np.float64)[:, :, b, None] * outs[b] for b in range(3))
+    g_lse = lse.cpu().numpy()
+    o_np = o.cpu().numpy()
+    for i in range(T):
+        dlt = o_np[i].astype(np.float64) - o_ref[i]
+        assert np.max(np.abs(dlt)) <= ATT_MAX_ABS, f"row {i}"
+        assert np.linalg.norm(dlt) <= ATT_REL_L2 * max(np.linalg.norm(o_ref[i]), 1e-30), f"row {i}"
+        for b in range(3):
+            fin = np.isfinite(lses[b][i])
+            assert np.array_equal(fin, np.isfinite(g_lse[b][i])), f"row {i} branch {b}: lse finiteness"
+            assert np.max(np.abs(g_lse[b][i][fin] - lses[b][i][fin])) <= ATT_MAX_ABS, f"row {i} branch {b}: lse"
+    # every surviving planted position's block is kept by its row's dynamic branch
+    for i in range(T):
+        p = c.plants[i][c.plants[i] >= 0]
+        assert np.isin(p // 128, g_blocks[i]).all(), f"row {i}: a planted block was dropped"
