@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -21,6 +22,7 @@
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
+#include "decode_fused.cuh"
 
 // Scratch of dsa_indexer_scores_noalloc: the query-tile plan for up to
 // DSA_NOALLOC_MAX_ROWS rows (about 256 KB).  Every device that loads this
@@ -57,6 +59,7 @@ struct DeviceState {
   bool probed = false;
   bool supported = false;
   bool prepared = false;
+  bool cooperative = false;
   int sm_count = 0;
   void* noalloc_plan = nullptr;  // device address of g_noalloc_plan on this device
 };
@@ -77,7 +80,11 @@ int current_device(DeviceState** out) {
         (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return cuda_fail(e, "cudaDeviceGetAttribute");
+    int coop = 0;
+    if ((e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
     d.supported = (major == 10 && minor == 0);
+    d.cooperative = coop != 0;
     d.sm_count = sms;
     d.probed = true;
   }
@@ -86,6 +93,7 @@ int current_device(DeviceState** out) {
     if ((e = dsa::prepare_indexer()) != cudaSuccess) return cuda_fail(e, "indexer smem opt-in");
     if ((e = dsa::prepare_sparse_mla()) != cudaSuccess) return cuda_fail(e, "sparse MLA smem opt-in");
     if ((e = dsa::prepare_topk()) != cudaSuccess) return cuda_fail(e, "top-k smem opt-in");
+    if ((e = dsa::prepare_decode_fused()) != cudaSuccess) return cuda_fail(e, "fused decode smem opt-in");
     d.prepared = true;
   }
   *out = &d;
@@ -198,10 +206,39 @@ dsa::StreamOut stream_out_at(uint8_t* sel, int T, int32_t* idx, int topk) {
   return so;
 }
 
-size_t ws_forward(int T, int64_t max_n_vis, int topk) {
+// The fused decode step (small batches): handoff counters and histograms, the
+// kept-position bitmaps and the candidate lists, after dsa_forward's own buffers.
+bool fused_fits(int T, int64_t max_n_vis) {
+  return T >= 1 && T <= dsa::kDecodeMaxRows && score_ld_for(max_n_vis) <= dsa::kDecodeMaxN;
+}
+struct FusedLayout {
+  size_t off_sync, off_cand, total;
+};
+FusedLayout fused_layout(size_t base, int T, int64_t max_n_vis) {
+  const int64_t ld = score_ld_for(max_n_vis);
+  FusedLayout L{};
+  L.off_sync = base;
+  L.off_cand = L.off_sync + align_up(dsa::decode_fused_sync_bytes(), 256);
+  L.total = L.off_cand + align_up(size_t(T) * size_t(ld) * 8, 256);
+  return L;
+}
+
+size_t ws_forward_base(int T, int64_t max_n_vis, int topk) {
   const size_t sel = forward_streams(T, max_n_vis) ? ws_select(T)
                                                    : align_up(size_t(T) * size_t(score_ld_for(max_n_vis)) * 4, 256);
   return ws_indexer(T) + sel + align_up(size_t(T) * size_t(topk) * 4, 256) + ws_mla(T, topk);
+}
+
+size_t ws_forward(int T, int64_t max_n_vis, int topk) {
+  const size_t base = ws_forward_base(T, max_n_vis, topk);
+  return fused_fits(T, max_n_vis) ? fused_layout(base, T, max_n_vis).total : base;
+}
+
+// DSA_DECODE_FUSED=1 runs small batches as the one-launch step (decode_fused.cuh);
+// by default they take the separate kernels, which are faster today.
+bool fused_enabled() {
+  const char* s = std::getenv("DSA_DECODE_FUSED");
+  return s && s[0] == '1';
 }
 
 // dense + sparse: window index rows (up to DSA_MAX_TOPK wide), the dense branch's
@@ -517,6 +554,44 @@ int dsa_forward(const dsa_bf16* q_I, const dsa_bf16* w, const dsa_bf16* k_I, con
   const int64_t ld = score_ld_for(max_n_vis);
   const bool streams = forward_streams(T, max_n_vis);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  // Small batches: one cooperative launch when every attention tile and every
+  // query's selection gets a CTA of its own.
+  if (fused_enabled() && !streams && dev->cooperative && fused_fits(T, max_n_vis) &&
+      int64_t(T) * ((std::min<int64_t>(topk, max_n_vis) + 127) / 128) + T <= dev->sm_count) {
+    const FusedLayout FL = fused_layout(ws_forward_base(T, max_n_vis, topk), T, max_n_vis);
+    uint8_t* sel0 = base + ws_indexer(T);
+    const size_t sel_bytes0 = align_up(size_t(T) * size_t(ld) * 4, 256);
+    int32_t* idx_ws0 = reinterpret_cast<int32_t*>(sel0 + sel_bytes0);
+    float* part0 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(idx_ws0) +
+                                            align_up(size_t(T) * size_t(topk) * 4, 256));
+    CUtensorMap tk, tqi, tq;
+    if ((rc = make_tmap_bf16(&tk, k_I, DSA_INDEX_DIM, uint64_t(cache_rows), 128))) return rc;
+    if ((rc = make_tmap_bf16(&tqi, q_I, DSA_INDEX_DIM, uint64_t(T) * DSA_INDEX_HEADS, 32))) return rc;
+    if ((rc = make_tmap_bf16(&tq, q, DSA_ROW, uint64_t(T) * DSA_HEADS, 64))) return rc;
+    dsa::DecodeFusedLaunch fp{};
+    fp.w = w;
+    fp.kv = kv;
+    fp.kv_start = kv_start;
+    fp.n_vis = n_vis;
+    fp.T = T;
+    fp.topk = topk;
+    fp.cache_rows = cache_rows;
+    fp.score_ld = ld;
+    fp.scale = scale;
+    fp.scores = reinterpret_cast<float*>(sel0);
+    fp.cand = base + FL.off_cand;
+    fp.sync = reinterpret_cast<uint32_t*>(base + FL.off_sync);
+    fp.part = part0;
+    fp.o_lat = o_lat;
+    fp.lse = lse;
+    fp.idx = idx_out ? idx_out : idx_ws0;
+    fp.sm_count = dev->sm_count;
+    fp.wait_ns = wait_limit_ns();
+    fp.stream = stream;
+    cudaError_t e = dsa::launch_decode_fused(fp, tk, tqi, tq);
+    if (e != cudaSuccess) return cuda_fail(e, "fused decode launch");
+    return DSA_OK;
+  }
   void* plan = base;
   uint8_t* sel = base + ws_indexer(T);  // score matrix, or the candidate buffers
   const size_t sel_bytes = streams ? ws_select(T) : align_up(size_t(T) * size_t(ld) * 4, 256);

@@ -292,7 +292,9 @@ __global__ void __launch_bounds__(idx_threads<QMAX>(), 1)
   constexpr int P = EPI / 4;              // epilogue warps per TMEM lane quarter
   constexpr int J = (QMAX + P - 1) / P;   // queries per epilogue warp (at most)
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KB-aligned base by pointer arithmetic on the shared array (an integer round trip
+  // would hide the shared address space and turn every access into a generic one)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   float* w_s = reinterpret_cast<float*>(smem + L::kWOff);
   int* nv_s = reinterpret_cast<int*>(smem + L::kNvOff);

@@ -122,10 +122,41 @@ cudaError_t launch_block_expand(const int32_t* blocks, const int32_t* n_vis, int
 cudaError_t launch_fuse3(float* o, const float* o_loc, const float* o_anc, const float* gates, int T, int sm_count,
                          cudaStream_t stream);
 
+// ------------------------------------------------------------------ fused decode step
+// The whole step of a batch of at most kDecodeMaxRows query rows in one
+// cooperative launch (one CTA per SM): indexer, exact top-k, attention, merge.
+constexpr int kDecodeMaxRows = 8;
+constexpr int kDecodeTileRows = 4;      // query rows per indexer tile
+constexpr int kDecodeMaxN = 32768;      // longest visible context (the row's scores sit in shared memory)
+struct DecodeFusedLaunch {
+  const uint16_t* w;
+  const uint16_t* kv;
+  const int64_t* kv_start;
+  const int32_t* n_vis;
+  int T;
+  int topk;
+  int64_t cache_rows;
+  int64_t score_ld;
+  float scale;
+  float* scores;      // [T, score_ld]
+  void* cand;         // [T, score_ld] pairs of (order key, position) that do not fit in shared memory
+  uint32_t* sync;     // handoff counters, zeroed before each launch
+  float* part;        // per attention tile: O (64 x 512), max, sum
+  float* o_lat;
+  float* lse;
+  int32_t* idx;
+  int sm_count;
+  unsigned long long wait_ns;
+  cudaStream_t stream;
+};
+cudaError_t launch_decode_fused(const DecodeFusedLaunch& p, const CUtensorMap& tmap_k, const CUtensorMap& tmap_qi,
+                                const CUtensorMap& tmap_q);
+
 // Shared-memory opt-in sizes, set once per device.
 cudaError_t prepare_indexer();
 cudaError_t prepare_sparse_mla();
 cudaError_t prepare_topk();
+cudaError_t prepare_decode_fused();
 // Exact top-k of each query's candidate buffer (after the streamed sweep),
 // written ascending and -1 padded; rows with cnt_out < 0 are left as they are.
 cudaError_t launch_stream_select(const StreamOut& so, const int32_t* n_vis, int T, cudaStream_t stream);

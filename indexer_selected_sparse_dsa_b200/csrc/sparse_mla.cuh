@@ -168,7 +168,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                       int topk, float scale_log2, float* __restrict__ o_lat, float* __restrict__ lse, int splits,
                       int tiles_per_split, float* __restrict__ part, WaitLimit lim) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1 KB-aligned base by pointer arithmetic on the shared array (an integer round trip
+  // would hide the shared address space and turn every access into a generic one)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   float* red = reinterpret_cast<float*>(smem + kRedOff);
   float* m_use = reinterpret_cast<float*>(smem + kMUseOff);

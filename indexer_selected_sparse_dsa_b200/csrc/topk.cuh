@@ -648,7 +648,7 @@ cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_
   const char* force = std::getenv("DSA_TOPK_KERNEL");
   const int force_full = (force && force[0] == 'r') ? 1 : 0;
   const bool force_short = force && force[0] == 's';
-  // Many short rows: three 256-thread CTAs per SM, one row each.
+  // Many short rows: one row per 256-thread CTA, as many CTAs per SM as the kernel's launch bound allows.
   if (!force_full && score_ld <= kShortMaxN && (force_short || T >= 2 * sm_count))
     return launch_pdl(topk_short_kernel, dim3(unsigned(T)), dim3(kShortThreads), sizeof(ShortShared), stream, 1,
                       scores, score_ld, n_vis, topk, idx);

@@ -15,7 +15,7 @@ from indexer_selected_sparse_dsa_b200 import binding as B
 from indexer_selected_sparse_dsa_b200 import workloads as wl
 
 from gpu_util import (ATT_MAX_ABS, ATT_REL_L2, SCALE, SET_TOL_REL, assert_attention_close, assert_scores_close,
-                      assert_selection_ok, gpu_attention, gpu_forward, gpu_scores, gpu_topk, to_dev)
+                      assert_selection_ok, gpu_attention, gpu_forward, gpu_scores, gpu_topk, reference_set, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -572,3 +572,120 @@ def test_block_sparse_matches_oracle(seed):
     for i in range(T):
         p = c.plants[i][c.plants[i] >= 0]
         assert np.isin(p // 128, g_blocks[i]).all(), f"row {i}: a planted block was dropped"
+
+
+# ---------------------------------------------------------------------------- fused decode step
+
+def _fused_case(name):
+    if name == "shared_cache_scaled":
+        return wl.make_workload_numpy(0, scale=4)
+    if name == "mixed_tiles":
+        # rows 0-3 share a sequence (one query tile), row 4 the same sequence (next tile),
+        # then one row per sequence; rows shorter and longer than topk
+        return wl.make_case_numpy([6000, 2048, 100, 3000],
+                                  [(0, 6000), (0, 5999), (0, 4000), (0, 2049), (0, 1), (1, 2048), (2, 100),
+                                   (3, 3000)], seed=71)
+    if name == "all_ties":
+        # every key of the second sequence is zero: its scores tie at 0 and the
+        # lowest positions win; the first sequence's keys take 5 values
+        c = wl.make_case_numpy([9000, 15000], [(0, 9000), (1, 15000), (1, 9000)], seed=72, n_plant=0)
+        c.k_I[9000:] = 0
+        c.k_I[:9000] = c.k_I[np.arange(9000) % 5]
+        return c
+    if name == "short_rows":
+        return wl.make_case_numpy([2048], [(0, 1), (0, 128), (0, 129), (0, 2048)], seed=73)
+    if name == "long_rows":  # the longest context the one-launch step takes
+        return wl.make_case_numpy([32768], [(0, 32768), (0, 30001)], seed=74)
+    raise KeyError(name)
+
+
+FUSED_CASES = ["shared_cache_scaled", "mixed_tiles", "all_ties", "short_rows", "long_rows"]
+
+
+@pytest.fixture
+def fused_on(monkeypatch):
+    monkeypatch.setenv("DSA_DECODE_FUSED", "1")
+
+
+@pytest.mark.parametrize("name", FUSED_CASES)
+def test_fused_decode_matches_oracle(name, fused_on):
+    """With DSA_DECODE_FUSED=1, dsa_forward on batches of at most 8 rows runs the one-launch decode step.
+    Its selection is checked bit-exactly against the oracle's top-k on the
+    kernel's own fp32 scores (read back from the workspace) and against fp64
+    scores within the tie band; the attention against the oracle on the
+    kernel's index set."""
+    import torch
+    c = _fused_case(name)
+    d = to_dev(c)
+    T, k = c.T, 2048
+    maxn = int(max(c.n_vis))
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    ws = B.workspace(B.DSA_OP_FORWARD, T, maxn, k)
+    B.dsa_forward(d["q_I"], d["w"], d["k_I"], d["q"], d["kv"], d["kv_start"], d["n_vis"], maxn, k, SCALE,
+                  o, lse, idx, ws)
+    B.dsa_sync_status()
+    ld = (maxn + 3) // 4 * 4
+    off = B.dsa_workspace_size(B.DSA_OP_INDEXER, T, maxn, k) // 4
+    S_gpu = ws.view(torch.float32)[off:off + T * ld].view(T, ld).cpu().numpy()
+    idx, o, lse = idx.cpu().numpy(), o.cpu().numpy(), lse.cpu().numpy()
+    S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=ld)
+    assert_scores_close(S_gpu, S_ref, c.n_vis)
+    S_own = np.where(np.arange(ld)[None, :] < c.n_vis[:, None], S_gpu, 0).astype(np.float64)
+    assert np.array_equal(idx, oracle.topk(S_own, c.n_vis, k)), "selection differs on the kernel's own scores"
+    assert_selection_ok(idx, S_ref, c.n_vis, k)
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+    for i in range(T):
+        p = c.plants[i][c.plants[i] >= 0]
+        assert np.isin(p, idx[i]).all(), f"row {i}: planted position dropped"
+    if name == "all_ties":
+        assert idx[1].tolist() == list(range(2048)) and idx[2].tolist() == list(range(2048))
+
+
+def test_fused_decode_skips_a_bad_row(fused_on):
+    import torch
+    c = wl.make_case_numpy([3000], [(0, 3000), (0, 2500), (0, 100)], seed=75)
+    d = to_dev(c)
+    d["n_vis"][1] = 5000                      # beyond the declared max_n_vis and the cache
+    T, k, maxn = 3, 2048, 3000
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((T, 64), float("nan"), dtype=torch.float32, device="cuda")
+    idx = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    ws = B.workspace(B.DSA_OP_FORWARD, T, maxn, k)
+    B.dsa_forward(d["q_I"], d["w"], d["k_I"], d["q"], d["kv"], d["kv_start"], d["n_vis"], maxn, k, SCALE,
+                  o, lse, idx, ws)
+    with pytest.raises(B.DSAError) as e:
+        B.dsa_sync_status()
+    assert e.value.code == B.DSA_ERR_BAD_ROW
+    idx, o, lse = idx.cpu().numpy(), o.cpu().numpy(), lse.cpu().numpy()
+    assert (idx[1] == -1).all() and (o[1] == 0).all() and np.isneginf(lse[1]).all()
+    good = [0, 2]
+    n_good = c.n_vis[good]
+    S_ref = oracle.indexer_scores(c.q_I[good], c.w[good], c.k_I, c.kv_start[good], n_good, score_ld=maxn)
+    assert_selection_ok(idx[good], S_ref, n_good, k)
+    o_ref, lse_ref = oracle.sparse_mla(c.q[good], c.kv, c.kv_start[good], idx[good], SCALE)
+    assert_attention_close(o[good], lse[good], o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("name", ["mixed_tiles", "long_rows"])
+def test_fused_and_separate_kernels_agree(name, monkeypatch):
+    """The one-launch step and the separate kernels select the same sets up to
+    near-ties (their fp32 head sums differ in order) and give the same attention."""
+    c = _fused_case(name)
+    d = to_dev(c)
+    maxn = int(max(c.n_vis))
+    monkeypatch.setenv("DSA_DECODE_FUSED", "1")
+    o_f, lse_f, idx_f = gpu_forward(d, maxn, 2048)
+    monkeypatch.setenv("DSA_DECODE_FUSED", "0")
+    o_s, lse_s, idx_s = gpu_forward(d, maxn, 2048)
+    S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, score_ld=maxn)
+    for i, n in enumerate(c.n_vis):
+        K = min(2048, int(n))
+        diff = np.setxor1d(idx_f[i, :K], idx_s[i, :K])
+        if diff.size:
+            _, kth = reference_set(S_ref[i, :n], K)
+            assert (np.abs(S_ref[i, diff] - kth) <= SET_TOL_REL * np.max(np.abs(S_ref[i, :n]))).all()
+        else:
+            assert np.max(np.abs(o_f[i] - o_s[i])) <= ATT_MAX_ABS
