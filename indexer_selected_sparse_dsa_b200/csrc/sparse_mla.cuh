@@ -553,50 +553,47 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
 // Merge the splits of each query row: with M = max_s m_s,
 //   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = (M + log2 of the denominator) * ln 2.
-// One CTA per (row, group of 4 heads): 2048 outputs, float4 loads of every split in flight.
-constexpr int kCombineHeads = 4;
+// One warp per (row, head, 128 latent dims): lane L owns dims 4 L .. 4 L + 3 and
+// has every split's float4 load in flight before the weights are known.
 constexpr int kCombineThreads = 256;
+constexpr int kCombineMaxSplits = 16;
 __global__ void __launch_bounds__(kCombineThreads) sparse_mla_combine_kernel(const float* __restrict__ part,
                                                                              int splits, float* __restrict__ o_lat,
                                                                              float* __restrict__ lse) {
-  __shared__ float wgt[16][kCombineHeads];
-  __shared__ float inv_den[kCombineHeads];
   pdl_wait();
-  const int groups = 64 / kCombineHeads;
-  const int i = blockIdx.x / groups;
-  const int h0 = (blockIdx.x - i * groups) * kCombineHeads;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int item = blockIdx.x * (kCombineThreads / 32) + warp;  // (row, head, quarter): the grid covers T x 256
+  const int i = item >> 8, h = (item >> 2) & 63, qd = item & 3;
   const float* p = part + (long long)i * splits * kPartFloats;
-  if (threadIdx.x < kCombineHeads) {
-    const int h = h0 + threadIdx.x;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmax_(M, p[(long long)s * kPartFloats + 64 * 512 + h]);
-    float den = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float ms = p[(long long)s * kPartFloats + 64 * 512 + h];
-      const float w = (M == -INFINITY) ? 0.f : fast_exp2(ms - M);
-      wgt[s][threadIdx.x] = w;
-      den += w * p[(long long)s * kPartFloats + 64 * 512 + 64 + h];
+  const int d = 128 * qd + 4 * lane;
+  float4 x[kCombineMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kCombineMaxSplits; ++s)
+    if (s < splits) x[s] = *reinterpret_cast<const float4*>(p + (long long)s * kPartFloats + h * 512 + d);
+  const float ms = lane < splits ? p[(long long)lane * kPartFloats + 64 * 512 + h] : -INFINITY;
+  const float ls = lane < splits ? p[(long long)lane * kPartFloats + 64 * 512 + 64 + h] : 0.f;
+  float M = ms;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmax_(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float w = (lane < splits && M > -INFINITY) ? fast_exp2(ms - M) : 0.f;
+  float den = w * ls;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s = 0; s < kCombineMaxSplits; ++s) {
+    const float ws = __shfl_sync(0xffffffffu, w, s);
+    if (s < splits) {
+      acc.x = fmaf(ws, x[s].x, acc.x);
+      acc.y = fmaf(ws, x[s].y, acc.y);
+      acc.z = fmaf(ws, x[s].z, acc.z);
+      acc.w = fmaf(ws, x[s].w, acc.w);
     }
-    inv_den[threadIdx.x] = den > 0.f ? 1.f / den : 0.f;
-    if (lse) lse[(long long)i * 64 + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
   }
-  __syncthreads();
-  const long long base = (long long)h0 * 512;
-  float* orow = o_lat + (long long)i * 64 * 512;
-  for (int v = threadIdx.x; v < kCombineHeads * 512 / 4; v += kCombineThreads) {
-    const int hl = (v * 4) >> 9;  // head within the group
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < splits; ++s) {
-      const float4 x = *reinterpret_cast<const float4*>(p + (long long)s * kPartFloats + base + v * 4);
-      const float w = wgt[s][hl];
-      acc.x = fmaf(w, x.x, acc.x);
-      acc.y = fmaf(w, x.y, acc.y);
-      acc.z = fmaf(w, x.z, acc.z);
-      acc.w = fmaf(w, x.w, acc.w);
-    }
-    const float id = inv_den[hl];
-    *reinterpret_cast<float4*>(orow + base + v * 4) = make_float4(acc.x * id, acc.y * id, acc.z * id, acc.w * id);
-  }
+  *reinterpret_cast<float4*>(o_lat + ((long long)i * 64 + h) * 512 + d) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lse && qd == 0 && lane == 0) lse[(long long)i * 64 + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace
@@ -630,8 +627,9 @@ cudaError_t launch_sparse_mla(const MlaLaunch& p, const CUtensorMap& tmap_q) {
                              p.kv, tmap_q, p.cache_rows, p.kv_start, p.idx, p.topk, scale_log2, p.o_lat, p.lse, splits,
                              per, p.part, WaitLimit{p.wait_ns});
   if (e != cudaSuccess || splits == 1) return e;
-  return launch_pdl(sparse_mla_combine_kernel, dim3(unsigned(p.T * (64 / kCombineHeads))), dim3(kCombineThreads), 0,
-                    p.stream, 1, p.part, splits, p.o_lat, p.lse);
+  static_assert(kMaxSplits <= kCombineMaxSplits, "the merge holds every split's load");
+  return launch_pdl(sparse_mla_combine_kernel, dim3(unsigned(p.T) * (256u / (kCombineThreads / 32))),
+                    dim3(kCombineThreads), 0, p.stream, 1, p.part, splits, p.o_lat, p.lse);
 }
 
 }  // namespace dsa
