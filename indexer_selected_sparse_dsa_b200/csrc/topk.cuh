@@ -555,10 +555,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
       cp_async_wait_all();
       m = gather_regions(kept0, reg_base, wcnt, sh);
       if (split > 1) {
-        // each CTA keeps at most its exact top-k (the union holds the row's);
-        // rank 0 then appends the other CTAs' lists through distributed
-        // shared memory, at most split * topk <= kCandCap entries
-        if (m > topk) {
+        // Rank 0 appends the other CTAs' lists through distributed shared memory
+        // and selects once over the union.  Each CTA sends every key that passed
+        // the shared threshold while its list fits its share of rank 0's buffer
+        // (the usual case: about 1.4 k / split keys each); a longer list is cut
+        // to its own exact top-k first (the union still holds the row's top-k).
+        if (m > kCandCap / split) {
           const Selection s = select_candidates(m, topk, sh);
           compact_kept(m, s, sh);
           m = topk;
@@ -660,7 +662,7 @@ cudaError_t launch_topk(const float* scores, int64_t score_ld, const int32_t* n_
     split = sm_count / T;
   }
   split = split >= 4 ? 4 : (split >= 2 ? 2 : 1);
-  static_assert(4 * DSA_MAX_TOPK <= kCandCap, "rank 0 holds every CTA's top-k");
+  static_assert(4 * DSA_MAX_TOPK <= kCandCap, "rank 0 holds every CTA's list (at most max(topk, kCandCap / split))");
   return launch_pdl(topk_kernel, dim3(unsigned(T) * unsigned(split)), dim3(kTopkThreads), sizeof(TopkShared), stream,
                     unsigned(split), scores, score_ld, n_vis, topk, idx, force_full, split);
 }
