@@ -29,9 +29,8 @@
 //     128B-swizzled layout, S^T = K.Q^T on the tensor cores (q was prefetched
 //     by TMA when the kernel started), the tile's softmax, O^T = V^T.P^T with
 //     P (bf16) written over the rope chunk the score product no longer needs.
-//     O goes through shared memory to global memory by bulk copy: the output
-//     itself for a one-tile query, else the tile's unnormalised O with its
-//     max and sum.
+//     O is stored from the registers the TMEM loads fill: the output itself
+//     for a one-tile query, else the tile's unnormalised O with its max and sum.
 //  -- handoff (only when a query has several tiles) --
 //  4. merge: one warp per (query, head, 128 latent dims) combines the tiles.
 // The selection follows the top-k kernels' rule (scores ranked by value, ties
@@ -67,8 +66,6 @@ constexpr int kFTileBytes = 9 * kFChunk;
 constexpr int kFKeyOff = kFTileOff;                               // 2 x 32 KB key stages
 constexpr int kFQiOff = kFKeyOff + kFStages * kFKeyStage;         // q_I tile: [half][4 queries] x 4 KB
 static_assert(kFQiOff + 2 * kDecodeTileRows * kFQiBox <= kFTileOff + kFTileBytes, "phase-1 buffers");
-// phase 3: the output staged in the tile region once the value product is done
-static_assert(kFPartFloats * 4 <= kFTileBytes, "output staging");
 // phase 2 (selection CTAs hold no attention tile: all of [0, kFMiscOff) is theirs):
 // the row's scores, its bitmap, the tie list, the window list (or, on the slow
 // path, one histogram per warp), the window histogram
@@ -78,6 +75,7 @@ constexpr int kFSelTieOff = kFSelBitmapOff + kDecodeMaxN / 8;     // 135168
 constexpr int kFSelTieCap = 256;
 constexpr int kFSelWinOff = 147456;
 constexpr int kFSelWinCap = 8192;                                 // (key, position) pairs (64 KB)
+constexpr int kFSelWinPerWarp = kFSelWinCap / kFWarps;            // each warp's region of the window list
 constexpr int kFSelWinHistOff = kFSelWinOff + kFSelWinCap * 8;    // 212992: 2048 bins
 // everything else
 constexpr int kFMiscOff = kFTileOff + kFTileBytes;  // 221184
@@ -142,24 +140,6 @@ __device__ __forceinline__ void warp_hist_add(uint32_t* hist, int bin, bool acti
   if (!active) return;
   const unsigned peers = __match_any_sync(act, bin);
   if ((threadIdx.x & 31) == __ffs(int(peers)) - 1) atomicAdd(&hist[bin], uint32_t(__popc(peers)));
-}
-
-// The key of rank r (1 = largest) among the warp's 256 keys (8 per lane): bitwise
-// radix from the top bit, one warp reduction per bit.
-__device__ __forceinline__ uint32_t warp_kth_largest(const uint32_t (&kv)[8], int r) {
-  uint32_t prefix = 0u, mask = 0u;
-#pragma unroll 1
-  for (int b = 31; b >= 0; --b) {
-    const uint32_t bit = 1u << b, want = prefix | bit, m2 = mask | bit;
-    int c = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) c += (kv[j] & m2) == want ? 1 : 0;
-    const int tot = int(__reduce_add_sync(0xffffffffu, unsigned(c)));
-    if (tot >= r) prefix = want;
-    else r -= tot;
-    mask = m2;
-  }
-  return prefix;
 }
 
 __device__ __forceinline__ uint32_t f_order_key(float x) {
@@ -545,74 +525,111 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (tid < 8) sel[tid] = 0;
       if (tid == 0 && !mbar_wait(sel_bar, 0, lim, abort_flag)) mbar_drain(sel_bar, 0);
       cta_sync();
-      // (b) a window [t_lo, t_hi] of order keys holding the k-th: each warp takes 256
-      //     strided scores and the keys of ranks r_lo and r_hi among them (exact, by a
-      //     bitwise radix over the warp); the CTA keeps the widest window
+      // (b) a window [t_lo, t_hi] of order keys holding the k-th: the keys of ranks
+      //     r_lo and r_hi among 2048 strided scores (exact: a bitwise radix over the
+      //     CTA, each warp counting its 256 samples, one warp reduction and one CTA
+      //     barrier per bit)
       uint32_t kv[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int si = warp * 256 + lane + 32 * j;
         kv[j] = f_order_key(sc[(int)((long long)si * n / (kFWarps * 256))]);
       }
-      const float sh = float(k) * 256.f / float(n);  // a warp sample's expected share of the top k
-      const int r_lo = min(256, int(ceilf(sh + 4.f * sqrtf(sh))) + 4);
-      const int r_hi = max(1, int(floorf(sh - 4.f * sqrtf(sh))) - 4);
-      const uint32_t lo_w = warp_kth_largest(kv, r_lo), hi_w = warp_kth_largest(kv, r_hi);
-      uint32_t* wlo = reinterpret_cast<uint32_t*>(red);  // red[] is idle in this phase
-      if (lane == 0) {
-        wlo[warp] = lo_w;
-        wlo[8 + warp] = hi_w;
-      }
-      cta_sync();
-      uint32_t t_lo = wlo[0], t_hi = wlo[8];
+      const float sh = float(k) * float(kFWarps * 256) / float(n);  // the sample's expected share of the top k
+      int r_lo = min(kFWarps * 256, int(ceilf(sh + 4.f * sqrtf(sh))) + 8);
+      int r_hi = max(1, int(floorf(sh - 4.f * sqrtf(sh))) - 8);
+      uint32_t t_lo = 0u, t_hi = 0u, mask = 0u;
+      int* bits_s = reinterpret_cast<int*>(red);  // [2 parities][8 warps][2 ranks]
+#pragma unroll 1
+      for (int b = 31; b >= 0; --b) {
+        const uint32_t bit = 1u << b, m2 = mask | bit, wa = t_lo | bit, wb = t_hi | bit;
+        int ca = 0, cb = 0;
 #pragma unroll
-      for (int w = 1; w < kFWarps; ++w) {
-        t_lo = min(t_lo, wlo[w]);
-        t_hi = max(t_hi, wlo[8 + w]);
+        for (int j = 0; j < 8; ++j) {
+          ca += (kv[j] & m2) == wa ? 1 : 0;
+          cb += (kv[j] & m2) == wb ? 1 : 0;
+        }
+        ca = int(__reduce_add_sync(0xffffffffu, unsigned(ca)));
+        cb = int(__reduce_add_sync(0xffffffffu, unsigned(cb)));
+        int* slot = bits_s + (b & 1) * 2 * kFWarps;
+        if (lane == 0) {
+          slot[2 * warp] = ca;
+          slot[2 * warp + 1] = cb;
+        }
+        __syncthreads();  // warps are converged here (every lane ran the reductions)
+        int ta = 0, tb = 0;
+#pragma unroll
+        for (int w = 0; w < kFWarps; ++w) {
+          ta += slot[2 * w];
+          tb += slot[2 * w + 1];
+        }
+        if (ta >= r_lo) t_lo = wa;
+        else r_lo -= ta;
+        if (tb >= r_hi) t_hi = wb;
+        else r_hi -= tb;
+        mask = m2;
       }
       const uint32_t span = t_hi - t_lo;
       const int shift = 32 - __clz(int(span >> 11));  // the smallest shift with (span >> shift) < 2048
-      // (c) one pass: keys above t_hi are kept; keys in the window go to its histogram and list
-      int gt = 0;
+      // (c) one pass, 4 consecutive positions per thread: keys above t_hi are kept
+      //     (bitmap words assembled from warp ballots, stored whole), keys in the
+      //     window are counted in its histogram and appended to the warp's region
+      //     of the window list (offsets from the ballots: no atomics, no scans)
+      int gt = 0, woff = 0;
+      const int wbase = warp * kFSelWinPerWarp;
+      auto spread4 = [](uint32_t m) {  // bit l of an 8-bit mask to bit 4 l
+        m = (m | (m << 12)) & 0x000F000Fu;
+        m = (m | (m << 6)) & 0x03030303u;
+        return (m | (m << 3)) & 0x11111111u;
+      };
       for (int base = 0; base < n4; base += 4 * kFThreads) {
         const int p0 = base + 4 * tid;
         uint32_t kk[4] = {0u, 0u, 0u, 0u};
-        int inw = 0;
         if (p0 < n4) {
           const float4 v = *reinterpret_cast<const float4*>(sc + p0);
           kk[0] = f_order_key(v.x);
           kk[1] = f_order_key(v.y);
           kk[2] = f_order_key(v.z);
           kk[3] = f_order_key(v.w);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (p0 + q >= n) continue;
-            if (kk[q] > t_hi) {
-              ++gt;
-              atomicOr(&bm[(p0 + q) >> 5], 1u << ((p0 + q) & 31));
-            } else if (kk[q] >= t_lo) {
-              ++inw;
-              atomicAdd(&wh[(kk[q] - t_lo) >> shift], 1u);
-            }
-          }
         }
-        const int inc = warp_inclusive_sum(inw);
-        int wb = 0;
-        if (lane == 31 && inc > 0) wb = atomicAdd(&sel[0], inc);
-        wb = __shfl_sync(0xffffffffu, wb, 31);
-        int slot = wb + inc - inw;
+        unsigned kb[4], wbl[4];
+        int wrun = 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (p0 + q < n && kk[q] <= t_hi && kk[q] >= t_lo) {
-            if (slot < kFSelWinCap) wl[slot] = make_uint2(kk[q], uint32_t(p0 + q));
-            ++slot;
+        for (int q = 0; q < 4; ++q) {
+          const bool valid = p0 + q < n;
+          const bool kept = valid && kk[q] > t_hi;
+          const bool inw = valid && !kept && kk[q] >= t_lo;
+          kb[q] = __ballot_sync(0xffffffffu, kept);
+          wbl[q] = __ballot_sync(0xffffffffu, inw);
+          gt += kept ? 1 : 0;
+          if (inw) {
+            const int slot = woff + wrun + __popc(wbl[q] & ((1u << lane) - 1u));
+            if (slot < kFSelWinPerWarp) wl[wbase + slot] = make_uint2(kk[q], uint32_t(p0 + q));
+            atomicAdd(&wh[(kk[q] - t_lo) >> shift], 1u);
           }
+          wrun += __popc(wbl[q]);
+        }
+        woff += wrun;
+        if (lane < 4) {  // word `lane` of the warp's 128 positions: lanes 8 lane .. 8 lane + 7
+          uint32_t word = 0u;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) word |= spread4((kb[q] >> (8 * lane)) & 0xFFu) << q;
+          const int wi = (base >> 5) + 4 * warp + lane;
+          if (wi < W) bm[wi] = word;
+        }
       }
+      if (lane == 0) sel[8 + warp] = woff;
       int gt_total = 0;
       (void)block_exclusive_sum<int>(gt, scan, &gt_total);
-      const int nw = sel[0];
+      int nw = 0;
+      bool fits = true;
+#pragma unroll
+      for (int w = 0; w < kFWarps; ++w) {
+        nw += sel[8 + w];
+        fits = fits && sel[8 + w] <= kFSelWinPerWarp;
+      }
       // (d) the window bin of the k-th key, counted from the top
-      bool ok = gt_total < k && gt_total + nw >= k && nw <= kFSelWinCap;
+      bool ok = fits && gt_total < k && gt_total + nw >= k;
       int bstar = 0, need = 0, eq = 0;
       {
         uint32_t cb[8];
@@ -643,7 +660,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
       ok = ok && eq <= kFSelTieCap;
       if (ok) {
         // (e) window keys above the bin are kept; the bin's keys go to the tie list
-        for (int j = tid; j < nw; j += kFThreads) {
+        for (int j = tid; j < kFWarps * kFSelWinPerWarp; j += kFThreads) {
+          if ((j % kFSelWinPerWarp) >= sel[8 + j / kFSelWinPerWarp]) continue;
           const uint2 e = wl[j];
           const int b = int((e.x - t_lo) >> shift);
           if (b > bstar) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
@@ -886,12 +904,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tc_fence_before();
     }
     cta_sync();
-    // O^T out of TMEM (warps 0-3: latent dims 0-255, warps 4-7: 256-511), staged as
-    // [head][512] floats (then the max and sum for a split row) and bulk-copied out
+    // O^T out of TMEM (warps 0-3: latent dims 0-255, warps 4-7: 256-511), stored as
+    // [head][512] floats (for a split row then its max and sum): a warp's store is
+    // 32 consecutive latent dims of one head
     if (*att_ok) {
       tc_fence_after();
       const bool single = R.tiles == 1;
-      float* st = reinterpret_cast<float*>(smem + kFTileOff);
+      float* dst = single ? a.o_lat + (long long)ra * 64 * 512 : a.part + (long long)blockIdx.x * kFPartFloats;
       const int qw = warp & 3;
       const uint32_t lane_addr = tmem + (uint32_t(qw * 32) << 16);
 #pragma unroll 1
@@ -905,7 +924,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
           for (int hh = 0; hh < 32; ++hh) {
             const int h = 32 * half + hh;
-            st[h * 512 + d] = single ? o[hh] / l_s[h] : o[hh];
+            dst[h * 512 + d] = single ? o[hh] / l_s[h] : o[hh];
           }
         }
       }
@@ -913,21 +932,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (single) {
           if (a.lse) a.lse[ra * 64 + tid] = (m_s[tid] + log2f(l_s[tid])) * 0.69314718055994531f;
         } else {
-          st[64 * 512 + tid] = m_s[tid];
-          st[64 * 512 + 64 + tid] = l_s[tid];
+          dst[64 * 512 + tid] = m_s[tid];
+          dst[64 * 512 + 64 + tid] = l_s[tid];
         }
-      }
-      fence_proxy_async_smem();
-      cta_sync();
-      if (tid == 0) {
-        float* dst = single ? a.o_lat + (long long)ra * 64 * 512 : a.part + (long long)blockIdx.x * kFPartFloats;
-        const uint32_t bytes = single ? 64 * 512 * 4 : kFPartFloats * 4;
-        for (uint32_t off = 0; off < bytes; off += 16384)
-          bulk_store_s2g(reinterpret_cast<uint8_t*>(dst) + off, sbase + kFTileOff + off,
-                         bytes - off < 16384 ? bytes - off : 16384);
-        bulk_commit();
-        bulk_wait_all();
-        fence_proxy_async_global();
       }
     }
   }
