@@ -111,7 +111,7 @@ constexpr int kFScanOff = (kFPlanOff + int(sizeof(FPlan)) + 15) & ~15;  // int s
 constexpr int kFSelOff = kFScanOff + 160;                               // int sel[16]
 constexpr int kFBarOff = (kFSelOff + 64 + 7) & ~7;
 constexpr int kFNumBars = 17;
-constexpr int kFSlotOff = kFBarOff + kFNumBars * 8;  // tmem slot, abort flag, phase-3 verdict
+constexpr int kFSlotOff = kFBarOff + kFNumBars * 8;  // tmem slot, abort flag, phase-3 outcome
 constexpr int kFSmemBytes = kFSlotOff + 16;
 constexpr int kFSmemAlloc = kFSmemBytes + 1024;
 constexpr uint32_t kFTmemCols = 512;

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 #pragma unroll
     for (int h = 0; h < 64; ++h) l_acc[h] = 0.f;
     // One softmax thread waits on the mbarrier; the barrier reduction then hands
-    // every softmax thread both the verdict and the memory ordering, so a failed
+    // every softmax thread both the outcome and the memory ordering, so a failed
     // wait ends the loop for all of them at the same point, before any named
     // barrier inside it.
     auto wait_all = [&](uint32_t bar, uint32_t parity) {

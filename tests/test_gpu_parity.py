@@ -596,10 +596,12 @@ def _fused_case(name):
         return wl.make_case_numpy([2048], [(0, 1), (0, 128), (0, 129), (0, 2048)], seed=73)
     if name == "long_rows":  # the longest context the one-launch step takes
         return wl.make_case_numpy([32768], [(0, 32768), (0, 30001)], seed=74)
+    if name == "eight_sequences":  # the largest batch: 8 query tiles of one row, 128 attention tiles
+        return wl.make_case_numpy([32768] * 8, [(b, 32768 - 1000 * b) for b in range(8)], seed=76)
     raise KeyError(name)
 
 
-FUSED_CASES = ["shared_cache_scaled", "mixed_tiles", "all_ties", "short_rows", "long_rows"]
+FUSED_CASES = ["shared_cache_scaled", "mixed_tiles", "all_ties", "short_rows", "long_rows", "eight_sequences"]
 
 
 @pytest.fixture
