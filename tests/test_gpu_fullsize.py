@@ -127,3 +127,55 @@ def test_full_size_workload(cfg, shard):
         o_ref, lse_ref = oracle.sparse_mla(a["q"], a["kv"], a["kv_start"], a["idx"], SCALE)
         assert_attention_close(run["o"][rb].cpu().numpy(), run["lse"][rb].cpu().numpy(), o_ref, lse_ref)
 
+
+
+# Block-level variant at the bench's size (bench.py --block-sparse: the 64-row, 128K
+# decode workload; 1024 blocks per row, 64 anchor blocks, 16 dynamic blocks): the
+# block choice on three rows equals the oracle's choice on the GPU's own fp32
+# scores, and the fused output and the three branches' lse match the oracle run on
+# those rows' own prefixes.
+BLOCK_ROWS = (0, 31, 63)
+
+
+def test_block_sparse_full_size_rows():
+    import torch
+    _RUN.clear()
+    torch.cuda.empty_cache()
+    from indexer_selected_sparse_dsa_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    c = wl.make_workload_torch(1, dev, seed=1)                 # same seed as bench.py rank 0
+    T = c.T
+    max_n = int(c.n_vis.max().item())
+    r = np.random.default_rng(77)
+    gates_h = r.uniform(0, 1, (T, 64, 3)).astype(np.float32)
+    gates = torch.from_numpy(gates_h).to(dev)
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device=dev)
+    lse = torch.full((3, T, 64), float("nan"), dtype=torch.float32, device=dev)
+    blocks = torch.full((T, oracle.BLOCK_TOPK), -7, dtype=torch.int32, device=dev)
+    ws = B.workspace(B.DSA_OP_BLOCK_SPARSE, T, max_n, 0, device=dev)
+    B.dsa_block_sparse_attn(c.q_I, c.w, c.k_I, c.q, c.kv, c.kv_start, c.n_vis, max_n, gates, SCALE, o, lse,
+                            blocks, ws)
+    B.dsa_sync_status()
+    ld = (max_n + 3) // 4 * 4
+    off = B.dsa_workspace_size(B.DSA_OP_INDEXER, T, max_n, 0)
+    rows = list(BLOCK_ROWS)
+    S_gpu = ws[off:off + T * ld * 4].view(torch.float32).view(T, ld)[rows].cpu().numpy()
+    h = host_rows(c, rows)
+    S_ref = oracle.indexer_scores(h["q_I"], h["w"], h["k_I"], h["kv_start"], h["n_vis"], score_ld=ld)
+    assert_scores_close(S_gpu, S_ref, h["n_vis"])
+    S_own = np.where(np.arange(ld)[None, :] < h["n_vis"][:, None], S_gpu, 0).astype(np.float64)
+    loc, anc, dyn, blk = oracle.block_branch_sets(S_own, h["n_vis"])
+    assert np.array_equal(blocks[rows].cpu().numpy(), blk), "block choice differs on the kernel's own scores"
+    g = gates_h[rows].astype(np.float64)
+    outs, lses = [], []
+    for idxs in (loc, anc, dyn):
+        o_b, lse_b = oracle.sparse_mla(h["q"], h["kv"], h["kv_start"], idxs, SCALE)
+        outs.append(o_b)
+        lses.append(lse_b)
+    o_ref = sum(g[:, :, b, None] * outs[b] for b in range(3))
+    lse_g = lse.cpu().numpy()
+    assert_attention_close(o[rows].cpu().numpy(), lse_g[2][rows], o_ref, lses[2])
+    for b in range(2):  # the local and anchor branches' lse
+        d = np.abs(lse_g[b][rows] - lses[b])
+        assert np.isfinite(lse_g[b][rows]).all() and d.max() <= 2e-2, (b, float(d.max()))

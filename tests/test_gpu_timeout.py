@@ -6,9 +6,10 @@ TMEM and exits; the call's status then reads DSA_ERR_TIMEOUT and the CUDA
 context stays usable.  A child process (so the test process never shares a
 context with an aborted kernel):
   1. runs the probe that waits on a barrier nothing completes: TIMEOUT;
-  2. runs the attention and the indexer with a 1 ns limit (their first wait
-     that is not already complete gives up): TIMEOUT, no CUDA error;
-  3. restores the default limit and runs both again in the same process:
+  2. runs the attention, the indexer and the one-launch decode step (its
+     grid-wide handoffs included) with a 1 ns limit (their first wait that is
+     not already complete gives up): TIMEOUT, no CUDA error;
+  3. restores the default limit and runs them again in the same process:
      status OK and the results match the oracle.
 """
 import json
@@ -30,7 +31,7 @@ sys.path.insert(0, ROOT)
 sys.path.insert(0, os.path.join(ROOT, "tests"))
 import oracle
 from indexer_selected_sparse_dsa_b200 import binding as B, build, workloads as wl
-from gpu_util import to_dev, assert_attention_close, assert_scores_close
+from gpu_util import to_dev, assert_attention_close, assert_scores_close, assert_selection_ok
 
 build.build()
 out = {}
@@ -60,18 +61,40 @@ def attention():
 def indexer():
     B.dsa_indexer_scores(d["q_I"], d["w"], d["k_I"], d["kv_start"], d["n_vis"], scores, ws_i)
 
+# the one-launch decode step (DSA_DECODE_FUSED=1): 3 rows over one 6000-position cache
+cf = wl.make_case_numpy([6000], [(0, 6000), (0, 5999), (0, 3000)], seed=12)
+df = to_dev(cf)
+of = torch.empty((3, 64, 512), device="cuda"); lsef = torch.empty((3, 64), device="cuda")
+idxf = torch.empty((3, k), dtype=torch.int32, device="cuda")
+ws_f = B.workspace(B.DSA_OP_FORWARD, 3, 6000, k)
+
+def fused():
+    os.environ["DSA_DECODE_FUSED"] = "1"
+    try:
+        B.dsa_forward(df["q_I"], df["w"], df["k_I"], df["q"], df["kv"], df["kv_start"], df["n_vis"], 6000, k,
+                      wl.SCALE, of, lsef, idxf, ws_f)
+    finally:
+        os.environ.pop("DSA_DECODE_FUSED", None)
+
 B.dsa_set_wait_limit_ns(2_000_000)                 # 2 ms: the probe gives up quickly
 out["probe"] = status_of(B.dsa_check_wait_timeout)
 B.dsa_set_wait_limit_ns(1)
 out["attention_1ns"] = status_of(attention)
 out["indexer_1ns"] = status_of(indexer)
+out["fused_1ns"] = status_of(fused)
 B.dsa_set_wait_limit_ns(0)                         # default limit again, same context
 out["attention_default"] = status_of(attention)
 out["indexer_default"] = status_of(indexer)
+out["fused_default"] = status_of(fused)
 o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, wl.SCALE)
 assert_attention_close(o.cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref)
 S_ref = oracle.indexer_scores(c.q_I, c.w, c.k_I, c.kv_start, c.n_vis, ld)
 assert_scores_close(scores.cpu().numpy(), S_ref, c.n_vis)
+idx_h = idxf.cpu().numpy()
+Sf = oracle.indexer_scores(cf.q_I, cf.w, cf.k_I, cf.kv_start, cf.n_vis, 6000)
+assert_selection_ok(idx_h, Sf, cf.n_vis, k)
+of_ref, lsef_ref = oracle.sparse_mla(cf.q, cf.kv, cf.kv_start, idx_h, wl.SCALE)
+assert_attention_close(of.cpu().numpy(), lsef.cpu().numpy(), of_ref, lsef_ref)
 out["parity_after"] = "OK"
 print("RESULT " + json.dumps(out), flush=True)
 '''
@@ -86,5 +109,7 @@ def test_bounded_waits_give_up_and_leave_the_context_usable():
     assert res["probe"] == "TIMEOUT", res
     assert res["attention_1ns"] == "TIMEOUT", res
     assert res["indexer_1ns"] == "TIMEOUT", res
+    assert res["fused_1ns"] == "TIMEOUT", res
     assert res["attention_default"] == "OK" and res["indexer_default"] == "OK", res
+    assert res["fused_default"] == "OK", res
     assert res["parity_after"] == "OK", res
