@@ -15,6 +15,8 @@ Two kinds of check on each workload's one run:
     of every surviving planted position.
 The oracle rows are split into shards so that no single test runs long.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -179,3 +181,48 @@ def test_block_sparse_full_size_rows():
     for b in range(2):  # the local and anchor branches' lse
         d = np.abs(lse_g[b][rows] - lses[b])
         assert np.isfinite(lse_g[b][rows]).all() and d.max() <= 2e-2, (b, float(d.max()))
+
+
+# NEXT rows at the bench's size (the 64-row, 128K decode workload), on the index
+# set dsa_forward selects: a shared layer of an IndexShare group (bench.py
+# --indexshare: its own queries and latent cache, the full layer's indices) and
+# the dense + sparse layer (bench.py --dense-window 512), each checked against the
+# oracle on three rows.
+NEXT_ROWS = (0, 33, 63)
+
+
+def test_indexshare_and_dense_sparse_full_size_rows():
+    import torch
+    run = _forward(1)
+    c, idx, T, k = run["c"], run["idx"], run["c"].T, run["k"]
+    dev = idx.device
+    rows = list(NEXT_ROWS)
+    g_idx = idx[rows].cpu().numpy()
+    # shared layer: its own q and kv, the full layer's idx
+    q1, kv1 = wl.make_shared_layer_torch(c, 1, dev, seed=1)
+    o1 = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device=dev)
+    l1 = torch.full((T, 64), float("nan"), dtype=torch.float32, device=dev)
+    ws_a = B.workspace(B.DSA_OP_SPARSE_MLA, T, 0, k, device=dev)
+    B.dsa_sparse_mla_attn(q1, kv1, c.kv_start, idx, SCALE, o1, l1, ws_a)
+    B.dsa_sync_status()
+    c1 = dataclasses.replace(c, q=q1, kv=kv1)
+    a = host_selected_rows(c1, rows, g_idx)
+    o_ref, lse_ref = oracle.sparse_mla(a["q"], a["kv"], a["kv_start"], a["idx"], SCALE)
+    assert_attention_close(o1[rows].cpu().numpy(), l1[rows].cpu().numpy(), o_ref, lse_ref)
+    del q1, kv1, c1
+    # dense + sparse: the last 512 visible positions and the selected set, fused per (row, head)
+    W = 512
+    gate_h = np.random.default_rng(78).uniform(0, 1, (T, 64)).astype(np.float32)
+    gate = torch.from_numpy(gate_h).to(dev)
+    o2 = torch.full((T, 64, 512), float("nan"), dtype=torch.float32, device=dev)
+    ld2 = torch.full((T, 64), float("nan"), dtype=torch.float32, device=dev)
+    ls2 = torch.full((T, 64), float("nan"), dtype=torch.float32, device=dev)
+    ws_d = B.workspace(B.DSA_OP_DENSE_SPARSE, T, 0, k, device=dev)
+    B.dsa_dense_sparse_attn(c.q, c.kv, c.kv_start, c.n_vis, idx, W, gate, SCALE, o2, ld2, ls2, ws_d)
+    B.dsa_sync_status()
+    h = host_rows(c, rows)
+    o_ref2, lsed_ref, lses_ref = oracle.dense_sparse(h["q"], h["kv"], h["kv_start"], h["n_vis"], g_idx, W,
+                                                     gate_h[rows], SCALE)
+    assert_attention_close(o2[rows].cpu().numpy(), ls2[rows].cpu().numpy(), o_ref2, lses_ref)
+    d = np.abs(ld2[rows].cpu().numpy() - lsed_ref)
+    assert d.max() <= 2e-2, float(d.max())
