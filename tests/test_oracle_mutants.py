@@ -72,3 +72,35 @@ def test_block_pins_catch_mutant(name, tmp_path):
         assert r.returncode == 0, r.stdout[-2000:]
     else:
         assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+# Plausible mistakes in the dense + sparse front end: the window shifted one
+# position back (the query no longer sees itself), the gate applied to the wrong
+# branch, the two branches' lse returned swapped.
+DENSE_MUTANTS = {
+    "window_shifted_back": ("p = n - window + np.arange(window", "p = n - window - 1 + np.arange(window"),
+    "gate_on_sparse_branch": ("return g * o_d + (1.0 - g) * o_s, lse_d, lse_s",
+                              "return g * o_s + (1.0 - g) * o_d, lse_d, lse_s"),
+    "branch_lse_swapped": ("return g * o_d + (1.0 - g) * o_s, lse_d, lse_s",
+                           "return g * o_d + (1.0 - g) * o_s, lse_s, lse_d"),
+}
+
+
+@pytest.mark.parametrize("name", ["unmutated"] + sorted(DENSE_MUTANTS))
+def test_dense_sparse_pins_catch_mutant(name, tmp_path):
+    old, new = DENSE_MUTANTS.get(name, ("", ""))
+    src = open(PY_SRC).read()
+    assert name == "unmutated" or src.count(old) == 1, name
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text((src.replace(old, new) if old else src).replace(
+        '_HERE = os.path.dirname(os.path.abspath(__file__))', '_HERE = %r' % os.path.join(ROOT, "oracle")))
+    env = dict(os.environ, PYTHONPATH=str(tmp_path) + os.pathsep + ROOT)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "-k", "dense_sparse",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=str(tmp_path), env=env, capture_output=True, text=True, timeout=600)
+    assert "passed" in r.stdout or "failed" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
+    if name == "unmutated":
+        assert r.returncode == 0, r.stdout[-2000:]
+    else:
+        assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
