@@ -16,12 +16,15 @@
 //     heads per key and writes the scores to the workspace.
 //  -- handoff --
 //  2. selection, one CTA per query (CTAs that hold no attention tile): the
-//     exact top-k of the query's scores in shared memory.  A histogram of the
-//     scores' 11-bit order-key prefixes (one copy per warp) gives the bin of
-//     the k-th score; scores above it are kept (a bitmap word per 32
-//     positions, set by warp ballots), those inside it become candidates,
-//     settled by a radix select over the remaining key bits and, for ties,
-//     over positions (the lower position wins).  The bitmap's popcount scan
+//     exact top-k of the query's scores, copied into shared memory.  The keys
+//     of two ranks among 2048 strided scores give a window of order keys that
+//     should hold the k-th score; one pass keeps the scores above the window
+//     (a bitmap word per 32 positions, built from warp ballots), and bins and
+//     lists those inside it; the bin of the k-th score is found by a scan and
+//     its few entries ranked by (score, lower position first).  When the
+//     window misses, an exact radix select over the whole row (per-warp
+//     histograms of 11-bit key prefixes, then the remaining key bits, then
+//     positions for ties) decides instead.  The bitmap's popcount scan
 //     writes the kept positions in ascending order (the idx output).
 //  -- handoff --
 //  3. attention, one CTA per (query, 128-position tile of its kept list):
