@@ -142,18 +142,20 @@ __device__ __forceinline__ void reduce_scatter64(const float (&v)[64], float& r0
   }
 }
 
-__device__ __forceinline__ int bar_red_or_128(int pred) {
+// bar.red.or over `nthreads` threads on named barrier `id`: 1 when any of them has pred != 0.
+__device__ __forceinline__ int bar_red_or(int id, int nthreads, int pred) {
   int out;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.s32 pi, %1, 0;\n\t"
-      "bar.red.or.pred po, 1, 128, pi;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
       "selp.s32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
-      : "r"(pred)
+      : "r"(pred), "r"(id), "r"(nthreads)
       : "memory");
   return out;
 }
+__device__ __forceinline__ int bar_red_or_128(int pred) { return bar_red_or(1, 128, pred); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& rlo, float& rhi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
@@ -268,10 +270,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       return (tile < ntiles && slot_i < topk) ? irow[slot_i] : -1;
     };
     int v0 = load_pos(0), v1 = load_pos(1);
-    for (int s = 0; s <= ntiles && ok; ++s) {
+    for (int s = 0; s <= ntiles; ++s) {
+      // Every producer is done reading y_s for the previous tile, and all of them
+      // agree whether to go on: a wait that failed in any one ends the loop for all
+      // (none is left behind at the named barrier below).
+      if (bar_red_or(2, 128, ok ? 0 : 1)) {
+        ok = false;
+        break;
+      }
       if (s < ntiles) {
         // cache rows of tile s (-1: empty or out of range) into y_s[s & 1]
-        named_bar_sync(2, 128);  // every producer is done reading this buffer's previous tile
         {
           int yy = -1;
           if (v0 >= 0) {

@@ -309,6 +309,20 @@ def test_attention_empty_row_and_large_logits(split):
     assert (o[1] == 0).all() and np.isneginf(lse[1]).all()
 
 
+def test_attention_more_rows_than_sms():
+    """More rows than SMs (several waves of CTAs); ragged lists of 1 to 384 keys."""
+    c = wl.make_case_numpy([1500], [(0, 1500)] * 300, seed=48, n_plant=0)
+    r = np.random.default_rng(48)
+    k = 384
+    idx = np.full((300, k), -1, np.int32)
+    for i in range(300):
+        m = [384, 200, 1, 257][i % 4]
+        idx[i, :m] = np.sort(r.choice(1500, m, replace=False))
+    o_ref, lse_ref = oracle.sparse_mla(c.q, c.kv, c.kv_start, idx, SCALE)
+    o, lse = gpu_attention(to_dev(c), idx, split=True)
+    assert_attention_close(o, lse, o_ref, lse_ref)
+
+
 def test_attention_per_row_cache_offsets():
     c = wl.make_case_numpy([700, 900, 300], [(0, 700), (1, 900), (2, 300), (1, 450)], seed=45, n_plant=0)
     r = np.random.default_rng(45)
