@@ -371,6 +371,23 @@ def test_forward_causal_prefill_short_rows():
             assert idx[i, :n].tolist() == list(range(n))
 
 
+def test_indexer_only_ranks():
+    """The indexer's scores decide which positions attend, never how much: doubling
+    w (exact in bf16) doubles every score exactly, and the selection, the output
+    and the lse stay the same bit for bit ("2026 LLM architecture overview (2):
+    DSA and MoE of GLM 5 / DSV3.2", section 2.2)."""
+    import torch
+    c = wl.make_case_numpy([6000] * 3, [(b, 6000 - 5 * b) for b in range(3)], seed=91)
+    d = to_dev(c)
+    o1, lse1, idx1 = gpu_forward(d, 6000, 2048)
+    d2 = dict(d)
+    d2["w"] = (d["w"].float() * 2).to(torch.bfloat16)
+    assert torch.equal(d2["w"].float(), d["w"].float() * 2)
+    o2, lse2, idx2 = gpu_forward(d2, 6000, 2048)
+    assert np.array_equal(idx1, idx2)
+    assert np.array_equal(o1, o2) and np.array_equal(lse1, lse2)
+
+
 def test_forward_ragged_decode_scaled():
     _forward_check(wl.make_workload_numpy(3, scale=32))
 
