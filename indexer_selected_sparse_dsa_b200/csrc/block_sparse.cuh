@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(32 * kBlockWarps) block_max_kernel(const float
                                                                      float* __restrict__ bscore,
                                                                      int32_t* __restrict__ nblocks) {
   pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.y;
   const int n = n_vis[i];
   const bool row_ok = n >= 1 && n <= score_ld && (n + kBlockTokens - 1) / kBlockTokens <= bld;
@@ -73,6 +74,7 @@ __global__ void block_expand_kernel(const int32_t* __restrict__ blocks, const in
                                     int wa, int32_t* __restrict__ idx_loc, int32_t* __restrict__ idx_anc,
                                     int32_t* __restrict__ idx_dyn) {
   pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x;
   const int n = n_vis[i];
   const int t = n - 1;  // n < 1: every list empty
@@ -102,6 +104,7 @@ __global__ void block_expand_kernel(const int32_t* __restrict__ blocks, const in
 __global__ void fuse3_kernel(float* __restrict__ o, const float* __restrict__ o_loc, const float* __restrict__ o_anc,
                              const float* __restrict__ gates, long long n4) {
   pdl_wait();
+  pdl_trigger();
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n4; v += (long long)gridDim.x * blockDim.x) {
     const float* g = gates + ((v * 4) >> 9) * 3;  // 512 latent dims per (row, head)
     const float gl = g[0], ga = g[1], gd = g[2];

@@ -23,6 +23,7 @@ namespace {
 // than the window); ascending, like every index row of the library.
 __global__ void window_idx_kernel(const int32_t* __restrict__ n_vis, int T, int window, int32_t* __restrict__ idx_w) {
   pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x;
   const int n = n_vis[i];
   if (n < 1 && threadIdx.x == 0) raise_status(kStatusBadRow);
@@ -37,6 +38,7 @@ __global__ void window_idx_kernel(const int32_t* __restrict__ n_vis, int T, int 
 __global__ void fuse_kernel(float* __restrict__ o, const float* __restrict__ o_dense, const float* __restrict__ gate,
                             long long n4) {
   pdl_wait();
+  pdl_trigger();
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n4; v += (long long)gridDim.x * blockDim.x) {
     const float g = gate[(v * 4) >> 9];  // 512 latent dims per (row, head)
     const float4 d = reinterpret_cast<const float4*>(o_dense)[v];

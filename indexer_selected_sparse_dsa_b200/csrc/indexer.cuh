@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(1024) indexer_plan_kernel(const int64_t* __res
   __shared__ int carry_seg_s;
   const int tid = threadIdx.x;
   pdl_wait();  // inputs and the plan buffer may belong to the previous kernel
+  pdl_trigger();
   for (int i = tid; i < T; i += blockDim.x) {
     PlanTile z;
     z.q0 = 0;
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(1024) indexer_redo_plan_kernel(const int* __re
                                                                  PlanTile* __restrict__ tiles) {
   __shared__ long long sc_l[33];
   pdl_wait();
+  pdl_trigger();
   const int n = redo[0];
   long long carry = 0;
   for (int base = 0; base < n; base += blockDim.x) {

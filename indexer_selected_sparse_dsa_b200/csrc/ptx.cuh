@@ -40,7 +40,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // (pdl_wait) before its first read of global memory another kernel may have
 // written; only shared-memory, TMEM and barrier setup come before the wait.
 // pdl_trigger lets the next kernel be scheduled once every CTA of this one has
-// triggered or exited.
+// triggered or exited; its CTAs then set up on free SMs and wait, and its wait
+// still returns only after this whole grid has finished and its writes are
+// visible.  The plan, top-k, selection and merge kernels trigger right after
+// their own wait (the next kernel's CTAs take SMs these leave idle); the
+// indexer and the attention, which hold every SM or TMEM, trigger at their end.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

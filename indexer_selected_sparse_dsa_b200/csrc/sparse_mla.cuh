@@ -569,6 +569,7 @@ __global__ void __launch_bounds__(kCombineThreads) sparse_mla_combine_kernel(con
                                                                              int splits, float* __restrict__ o_lat,
                                                                              float* __restrict__ lse) {
   pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int item = blockIdx.x * (kCombineThreads / 32) + warp;  // (row, head, quarter): the grid covers T x 256
   const int i = item >> 8, h = (item >> 2) & 63, qd = item & 3;

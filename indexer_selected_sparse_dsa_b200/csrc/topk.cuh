@@ -413,6 +413,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
   pdl_wait();  // the scores come from the previous kernel
+  pdl_trigger();
   // `split` CTAs (one cluster) per row; every branch below that returns early
   // depends on the row alone, so a cluster's CTAs take it together
   const int r = blockIdx.x / split;
@@ -609,6 +610,7 @@ __global__ void __launch_bounds__(kTopkThreads) stream_select_kernel(const uint3
   extern __shared__ __align__(16) uint8_t topk_smem[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(topk_smem);
   pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int m = min(cnt[r], cap);
   if (m < 0) return;

@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(kShortThreads, 5)
   extern __shared__ __align__(16) uint8_t short_smem[];
   ShortShared& sh = *reinterpret_cast<ShortShared*>(short_smem);
   pdl_wait();  // the scores come from the previous kernel
+  pdl_trigger();
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31;
   const int n = n_vis[r];
