@@ -1,16 +1,20 @@
 """Benchmark of the DSA sparse-attention step (indexer -> top-k -> sparse MLA).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config C] [--scale S] [--skip-cpu] [--skip-e2e] [--indexshare L]
-                    [--dense-window W]
+                    [--config C] [--scale S] [--skip-cpu] [--skip-e2e] [--e2e-serial]
+                    [--workloads auto|none|LIST] [--no-graph] [--indexshare L]
+                    [--dense-window W] [--block-sparse]
 
 One step = one dsa_forward over one batch of the workload (every query row:
 indexer over its causal context, exact top-2048, sparse latent MLA).  The
 default workload is batch-64 decode at 131072 context per sequence.  Inputs
-are synthetic (seeded) and resident in HBM; the per-step working set (about
-2.3 GB) is far larger than the 126 MB L2, so no L2 flush is needed between
-steps.  Under torchrun every rank runs its own batch (weak scaling; the
-path has no data exchange between rows).  Rank 0 prints one JSON line.
+are synthetic (seeded) and resident in HBM; the default per-step working set
+(about 2.3 GB) is far larger than the 126 MB L2, so no L2 flush is needed
+between its steps (a workload whose inputs fit in L2 is flushed before every
+timed step and its steps are timed one by one).  The line's `workloads` key
+carries the other workloads, each timed for about a second.  Under torchrun
+every rank runs its own batch (weak scaling; the path has no data exchange
+between rows).  Rank 0 prints one JSON line.
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload shape
 (rank 0 only; bounded samples of query rows per step).
